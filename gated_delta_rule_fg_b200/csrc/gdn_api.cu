@@ -1,0 +1,172 @@
+// gdn_api.cu -- the C ABI declared in include/gdn.h: argument validation,
+// workspace sizing and kernel dispatch.  Every step of the computation runs in
+// the CUDA kernels of this library; there is no host or CPU fallback.
+#include "gdn.h"
+#include "gdn_common.cuh"
+
+namespace gdn {
+// gdn_simt.cu
+size_t simt_inter_bytes(const Problem& p);
+bool simt_supported(int C, int dk, int dv);
+cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream);
+// gdn_tc.cu
+bool tc_supported(const Problem& p, bool bf16);
+size_t tc_inter_bytes(const Problem& p);
+cudaError_t launch_tc(const Problem& p, cudaStream_t stream);
+int tc_launches(const Problem& p);
+}  // namespace gdn
+
+using namespace gdn;
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;     // status word + reserved, keeps the rest 256-aligned
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+// Fills `p` (without pointers) and checks sizes.  Returns GDN_OK or the error.
+gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int dv, int chunk,
+                          gdn_dtype_t dtype, unsigned flags, bool dp) {
+    if (B < 0 || H < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR)) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+    if (dp && (nh < 1 || nh > 4)) return GDN_ERR_UNSUPPORTED;
+    const bool beta_scalar = dp || (flags & GDN_BETA_SCALAR);
+    if (!beta_scalar && dk != dv) return GDN_ERR_INVALID_ARG;
+    if (!simt_supported(chunk, dk, dv)) return GDN_ERR_UNSUPPORTED;
+    p = Problem{};
+    p.B = B; p.H = H; p.T = T;
+    p.nh = dp ? nh : 1;
+    p.L = T * p.nh;
+    p.dk = dk; p.dv = dv; p.C = chunk;
+    p.NC = (p.L + chunk - 1) / chunk;
+    p.alpha_scalar = dp ? 1 : ((flags & GDN_ALPHA_SCALAR) ? 1 : 0);
+    p.beta_scalar = beta_scalar ? 1 : 0;
+    p.dp = dp ? 1 : 0;
+    return GDN_OK;
+}
+
+size_t workspace_bytes_for(const Problem& p, bool bf16) {
+    size_t inter = tc_supported(p, bf16) ? tc_inter_bytes(p) : simt_inter_bytes(p);
+    return kHeaderBytes + inter;
+}
+
+gdn_status_t run(Problem& p, bool bf16, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+    const bool has_tokens = p.B > 0 && p.H > 0 && p.T > 0;
+    if (has_tokens && (!p.q || !p.k || !p.v || !p.alpha || !p.beta || !p.out)) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.alpha) ||
+        !aligned16(p.beta) || !aligned16(p.out) || !aligned16(p.S0) || !aligned16(p.S_final))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = workspace_bytes_for(p, bf16);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return GDN_ERR_WORKSPACE;
+    p.status = static_cast<int*>(workspace);
+    p.inter = static_cast<char*>(workspace) + kHeaderBytes;
+    if (p.B == 0 || p.H == 0) return GDN_OK;
+    cudaError_t e = tc_supported(p, bf16) ? launch_tc(p, stream) : launch_simt(p, bf16, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+int launches_for(const Problem& p, bool bf16) {
+    if (p.B == 0 || p.H == 0) return 0;
+    if (tc_supported(p, bf16)) return tc_launches(p);
+    return p.NC > 0 ? 2 : 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                           unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false) != GDN_OK) return -1;
+    return launches_for(p, dtype == GDN_BF16);
+}
+
+int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype) {
+    Problem p;
+    if (make_problem(p, B, H, T, n_h, dk, dv, chunk, dtype, 0u, true) != GDN_OK) return -1;
+    return launches_for(p, dtype == GDN_BF16);
+}
+
+size_t gdn_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                    gdn_dtype_t dtype, unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false) != GDN_OK) return 0;
+    return workspace_bytes_for(p, dtype == GDN_BF16);
+}
+
+gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta,
+                           const float* S0, void* out, float* S_final,
+                           int B, int H, int T, int dk, int dv, int chunk,
+                           gdn_dtype_t dtype, unsigned flags,
+                           void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+    Problem p;
+    gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false);
+    if (st != GDN_OK) return st;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta;
+    p.S0 = S0; p.out = out; p.S_final = S_final;
+    return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
+}
+
+size_t gdn_deltaproduct_fwd_workspace_size(int B, int H, int T, int n_h, int dk, int dv,
+                                           int chunk, gdn_dtype_t dtype) {
+    Problem p;
+    if (make_problem(p, B, H, T, n_h, dk, dv, chunk, dtype, 0u, true) != GDN_OK) return 0;
+    return workspace_bytes_for(p, dtype == GDN_BF16);
+}
+
+gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
+                                  const float* gamma, const float* beta,
+                                  const float* S0, void* out, float* S_final,
+                                  int B, int H, int T, int n_h, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype,
+                                  void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+    Problem p;
+    gdn_status_t st = make_problem(p, B, H, T, n_h, dk, dv, chunk, dtype, 0u, true);
+    if (st != GDN_OK) return st;
+    p.q = q; p.k = k; p.v = v; p.alpha = gamma; p.beta = beta;
+    p.S0 = S0; p.out = out; p.S_final = S_final;
+    return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
+}
+
+gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream) {
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GDN_ERR_CUDA;
+    if (word != 0 && cudaMemset(workspace, 0, sizeof(int)) != cudaSuccess) return GDN_ERR_CUDA;
+    switch (word) {
+        case 0: return GDN_OK;
+        case kDevTimeout: return GDN_ERR_TIMEOUT;
+        case kDevRange: return GDN_ERR_RANGE;
+        default: return GDN_ERR_CUDA;
+    }
+}
+
+const char* gdn_status_string(gdn_status_t s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported size";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "device wait timed out";
+        case GDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case GDN_ERR_RANGE: return "value outside the fp16 operand range";
+    }
+    return "unknown status";
+}
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

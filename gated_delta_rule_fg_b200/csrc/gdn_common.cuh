@@ -1,0 +1,98 @@
+// gdn_common.cuh -- problem description and helpers shared by the kernels of
+// libgdn_b200.so.
+//
+// The chunkwise evaluation of the FG^2-GDN recurrence (reading notes of
+// "FG^2-GDN: Enhancing Long-Context Gated Delta Networks with Doubly
+// Fine-Grained Control", sec. 2.2 eq. (11) and sec. 2.4) is split in two roles:
+//
+//   intra role (independent per chunk): load a chunk of C rows, L2-normalise
+//     q and k, scale k and v by sqrt(beta), take the cumulative log-decay
+//     g_r = sum_{s<=r} log alpha_s per channel, and build
+//       A   = strictly-lower (K~ e^g)(K~ e^-g)^T    P = lower (Q^ e^g)(K~ e^-g)^T
+//       T   = (I + A)^{-1}                          (UT transform)
+//       W   = T (K~ (.) e^g)        U'  = T V~
+//       Qe  = Q^ (.) e^g - P W      PU' = P U'
+//       K'  = K~ (.) e^{g_C - g}    gC  = e^{g_C}
+//   scan role (serial over chunks, per head and d_v slice), with S the state
+//     at the chunk start:
+//       U = U' - W S;   O = Qe S + PU';   S <- Diag(gC) S + K'^T U
+//
+// The scan-role formulas follow from eq. (11): with X_r = Diag(alpha_r) S_{r-1}
+// and u_r = v~_r - X_r^T k~_r, (I + A) U = V~ - (K~ (.) e^g) S, the outputs are
+// O = (Q^ (.) e^g) S + P U and the next state is Diag(e^{g_C}) S + K'^T U;
+// substituting U = U' - W S into O gives O = Qe S + PU'.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Device-side error codes recorded in the workspace header (match gdn_status_t).
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevRange = 6 };
+
+struct Problem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;     // GDN: alpha; DeltaProduct: gamma (scalar per token)
+    const float* beta;
+    const float* S0;        // may be null
+    void* out;
+    float* S_final;         // may be null
+    int B, H, T;            // T = tokens
+    int nh;                 // sub-steps per token (1 for GDN, n_h for DeltaProduct)
+    int L;                  // sub-steps per sequence = T * nh
+    int dk, dv, C;          // head dims and chunk length (in sub-steps)
+    int NC;                 // chunks per sequence = ceil(L / C)
+    int alpha_scalar, beta_scalar;
+    int dp;                 // 1: DeltaProduct row mapping
+    int* status;            // workspace header word
+    void* inter;            // per-chunk intermediates written by the intra role
+};
+
+// Row source of sub-step s of head (b, h) (DeltaProduct interleaves n_h
+// sub-steps per token; the decay gamma_t sits on the first one and the output
+// is read at the last one).
+struct RowRef {
+    size_t tok;        // (b*T + t)*H + h
+    int m;             // sub-step within the token
+    bool has_q;        // this row produces an output
+};
+
+__device__ __forceinline__ RowRef row_ref(const Problem& p, int b, int h, int s) {
+    RowRef r;
+    int t = s / p.nh;
+    r.m = s - t * p.nh;
+    r.tok = ((size_t)b * p.T + t) * p.H + h;
+    r.has_q = (r.m == p.nh - 1);
+    return r;
+}
+
+__device__ __forceinline__ float load_in(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_in(const __nv_bfloat16* p, size_t i) { return __bfloat162float(p[i]); }
+__device__ __forceinline__ void store_out(float* p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_out(__nv_bfloat16* p, size_t i, float x) { p[i] = __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+constexpr float kNormEps = 1e-6f;   // ||x|| = sqrt(sum x^2 + eps)
+
+// Layout of the float32 intermediates of one (head, chunk) in the workspace.
+struct InterF32 {
+    int C, dk, dv;
+    __host__ __device__ size_t floats() const { return (size_t)C * (3 * dk + 2 * dv) + dk; }
+    __host__ __device__ size_t W() const { return 0; }
+    __host__ __device__ size_t Qe() const { return (size_t)C * dk; }
+    __host__ __device__ size_t Kp() const { return 2 * (size_t)C * dk; }
+    __host__ __device__ size_t Up() const { return 3 * (size_t)C * dk; }
+    __host__ __device__ size_t PUp() const { return 3 * (size_t)C * dk + (size_t)C * dv; }
+    __host__ __device__ size_t gC() const { return 3 * (size_t)C * dk + 2 * (size_t)C * dv; }
+};
+
+}  // namespace gdn

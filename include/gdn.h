@@ -1,0 +1,152 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) FG^2-GDN chunkwise forward library
+ *          (libgdn_b200.so).
+ *
+ * The operation.  For every (batch b, head h) pair the library evaluates the
+ * FG^2-GDN recurrence ("FG^2-GDN: Enhancing Long-Context Gated Delta Networks
+ * with Doubly Fine-Grained Control", sec. 2 "FG2-GDN Update Rule"; reading
+ * notes of the same paper, sec. 2.2, eq. (11)):
+ *
+ *     q^_t = q_t / ||q_t||,   k^_t = k_t / ||k_t||     (||x|| = sqrt(sum x^2 + 1e-6))
+ *     k~_t = sqrt(beta_t) (.) k^_t,   v~_t = sqrt(beta_t) (.) v_t
+ *     S_t  = (I - k~_t k~_t^T) Diag(alpha_t) S_{t-1} + k~_t v~_t^T
+ *     o_t  = S_t^T q^_t
+ *
+ * with S in R^{dk x dv}, channel-wise decay alpha_t in (0,1]^{dk} and
+ * channel-wise write rate beta_t in [0,1]^{dk}.  KDA (scalar beta), GDN
+ * (scalar alpha and beta) and DeltaNet (alpha = 1, scalar beta) are the special
+ * cases selected with GDN_ALPHA_SCALAR / GDN_BETA_SCALAR (reading notes, sec. 1
+ * table).  It is computed chunkwise: the sequence is cut into chunks of
+ * `chunk` tokens, the transitions inside a chunk are accumulated in parallel
+ * through the WY/UT representation (cumulative log-decay per chunk, a
+ * strictly lower-triangular (I + A)^{-1} solve), and the state is carried from
+ * chunk to chunk (reading notes, sec. 2.4).  The result does not depend on
+ * `chunk` beyond rounding.
+ *
+ * Conventions shared by every entry point.
+ *   - All tensor arguments are device pointers, row-major and contiguous,
+ *     owned by the caller; the library never frees or retains them.
+ *   - q, k: [B,T,H,dk]; v, out: [B,T,H,dv]; alpha, beta: [B,T,H,dk], or
+ *     [B,T,H] with GDN_ALPHA_SCALAR / GDN_BETA_SCALAR; S0, S_final:
+ *     [B,H,dk,dv] float32.
+ *   - q, k, v and out share one storage type (gdn_dtype_t).  alpha, beta and
+ *     the state are always float32.  Arithmetic is float32 (GDN_F32) or
+ *     bf16 inputs with fp16 tensor-core operands and float32 accumulation and
+ *     state (GDN_BF16); `out` is rounded to nearest-even on store.
+ *   - alpha and beta are post-activation values.  Values outside alpha in
+ *     (0,1], beta >= 0, or NaN are not checked (that would cost a pass over
+ *     the inputs) and give undefined numbers, not an error.
+ *   - S0 == NULL means a zero initial state; S_final == NULL means the final
+ *     state is not written.  Feeding S_final back as S0 continues a sequence.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns once it is enqueued.  The caller provides
+ *     `workspace` (device memory, 256-byte aligned, at least the size the
+ *     matching *_workspace_size function returns); one workspace must not be
+ *     used by two calls that can run at the same time.  The library allocates
+ *     nothing and keeps no global state.
+ *   - Arguments are validated before anything is enqueued; on an error
+ *     nothing is enqueued.  Errors found on the device (a bounded wait that
+ *     ran out, a value outside the fp16 operand range) are recorded in the
+ *     workspace and read with gdn_workspace_status().
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* NULL / misaligned pointer, negative size, dk != dv with channel-wise beta */
+    GDN_ERR_UNSUPPORTED = 2,   /* a size this build does not implement (see gdn_chunk_fwd) */
+    GDN_ERR_CUDA = 3,          /* a CUDA launch or copy failed (cudaGetLastError is left set) */
+    GDN_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out; outputs are not valid */
+    GDN_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or smaller than required */
+    GDN_ERR_RANGE = 6          /* device side: a state or value exceeded the fp16 operand range */
+} gdn_status_t;
+
+typedef enum {
+    GDN_F32 = 0,               /* q, k, v, out stored as float32 */
+    GDN_BF16 = 1               /* q, k, v, out stored as bfloat16 */
+} gdn_dtype_t;
+
+enum {
+    GDN_ALPHA_SCALAR = 1u,     /* alpha is one value per token and head: [B,T,H] (GDN) */
+    GDN_BETA_SCALAR = 2u       /* beta is one value per token and head: [B,T,H] (KDA, GDN, DeltaNet) */
+};
+
+/* Bytes of workspace gdn_chunk_fwd needs for these sizes (0 if the sizes are
+ * invalid or unsupported; gdn_chunk_fwd then reports why). */
+size_t gdn_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                    gdn_dtype_t dtype, unsigned flags);
+
+/* FG^2-GDN chunkwise forward (eq. (11) above).
+ *   q, k [B,T,H,dk], v [B,T,H,dv], out [B,T,H,dv]: dtype storage.
+ *   alpha, beta: float32, channel-wise or scalar per `flags`.
+ *   S0 (may be NULL), S_final (may be NULL): float32 [B,H,dk,dv].
+ * Sizes: B, H, T >= 0 (zero is a no-op that still writes S_final = S0 or 0;
+ * with T == 0 the token pointers may be NULL); dk, dv in {32, 64, 128};
+ * chunk in {16, 32, 64}.  Channel-wise beta needs dk == dv (sqrt(beta) multiplies v).
+ * T need not be a multiple of chunk.  GDN_BF16 with chunk == 64 and
+ * dk == dv == 128 runs on the tensor-core path; other GDN_BF16 shapes and all
+ * GDN_F32 shapes run on the float32 CUDA-core path. */
+gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta,
+                           const float* S0, void* out, float* S_final,
+                           int B, int H, int T, int dk, int dv, int chunk,
+                           gdn_dtype_t dtype, unsigned flags,
+                           void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* Bytes of workspace gdn_deltaproduct_fwd needs (0 if invalid/unsupported). */
+size_t gdn_deltaproduct_fwd_workspace_size(int B, int H, int T, int n_h, int dk, int dv,
+                                           int chunk, gdn_dtype_t dtype);
+
+/* DeltaProduct n_h forward with a scalar forget gate ("DeltaProduct: Improving
+ * State-Tracking in Linear RNNs via Householder Products", "Approach"; the
+ * gated variant of its ablation table).  Per token t:
+ *     S <- gamma_t S;  for m = 1..n_h:  S <- (I - beta_{t,m} k^_{t,m} k^_{t,m}^T) S
+ *                                             + beta_{t,m} k^_{t,m} v_{t,m}^T
+ *     o_t = S^T q^_t
+ * (gamma is applied once per token, before the first step; k^ and q^ are
+ * L2-normalised as above; beta in [0,2] gives eigenvalues in [-1,1]).  It is
+ * evaluated as the FG^2-GDN recurrence over the interleaved sequence of n_h*T
+ * sub-steps with scalar beta; `chunk` counts sub-steps.
+ *   q [B,T,H,dk]; k [B,T,H,n_h,dk]; v [B,T,H,n_h,dv]; gamma [B,T,H];
+ *   beta [B,T,H,n_h]; S0, S_final [B,H,dk,dv] float32; out [B,T,H,dv].
+ * Sizes as gdn_chunk_fwd, with 1 <= n_h <= 4. */
+gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
+                                  const float* gamma, const float* beta,
+                                  const float* S0, void* out, float* S_final,
+                                  int B, int H, int T, int n_h, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype,
+                                  void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
+/* Number of kernels one gdn_chunk_fwd / gdn_deltaproduct_fwd call with these
+ * sizes enqueues (-1 if the sizes are invalid or unsupported). */
+int gdn_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                           unsigned flags);
+int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype);
+
+/* Waits for `stream`, then returns (and clears) the first device-side error
+ * recorded in `workspace` by earlier calls: GDN_OK, GDN_ERR_TIMEOUT or
+ * GDN_ERR_RANGE; GDN_ERR_CUDA if the wait itself failed. */
+gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* gdn_status_string(gdn_status_t status);
+
+/* Library ABI version (major * 100 + minor). */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_B200_H */

@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+symbol include/gdn.h declares, sizes the workspace, and validates arguments before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_fg_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+FAKE = 0x10000            # an aligned, never dereferenced stand-in for a device pointer
+FAKE_ODD = 0x10008        # 8-byte aligned only
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_fg_b200 import build
+    build.build()
+    return ops.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"gdn_chunk_fwd", "gdn_deltaproduct_fwd", "gdn_workspace_status"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in gdn.h but not exported"
+        assert n in ops.SIGNATURES, f"{n} has no ctypes signature in ops.py"
+
+
+def test_version_and_status_strings(L):
+    assert L.gdn_version() >= 100
+    for code in range(7):
+        assert len(ops.status_string(code)) > 0
+    assert ops.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(L):
+    ws = ops.chunk_fwd_workspace_size
+    assert ws(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) > 0
+    assert ws(1, 2, 256, 32, 32, 16, ops.GDN_F32, 0) > 0
+    assert ws(1, 1, 0, 64, 64, 64, ops.GDN_F32, 0) > 0          # T = 0 is valid
+    assert ws(1, 1, 10, 48, 48, 64, ops.GDN_F32, 0) == 0        # unsupported head dim
+    assert ws(1, 1, 10, 64, 64, 48, ops.GDN_F32, 0) == 0        # unsupported chunk
+    assert ws(1, 1, 10, 64, 128, 64, ops.GDN_F32, 0) == 0       # channel-wise beta, dk != dv
+    assert ws(1, 1, 10, 64, 128, 64, ops.GDN_F32, ops.GDN_BETA_SCALAR) > 0
+    assert ws(-1, 1, 10, 64, 64, 64, ops.GDN_F32, 0) == 0
+    a = ws(1, 4, 1000, 64, 64, 32, ops.GDN_F32, 0)
+    b = ws(1, 4, 2000, 64, 64, 32, ops.GDN_F32, 0)
+    assert b > a                                                # grows with T
+    dws = ops.deltaproduct_fwd_workspace_size
+    assert dws(2, 8, 8192, 2, 128, 128, 64, ops.GDN_BF16) > 0
+    assert dws(2, 8, 8192, 5, 128, 128, 64, ops.GDN_BF16) == 0  # n_h > 4
+
+
+def _call(L, q=FAKE, k=FAKE, v=FAKE, alpha=FAKE, beta=FAKE, S0=None, out=FAKE, Sf=None,
+          B=1, H=1, T=8, dk=64, dv=64, chunk=64, dtype=ops.GDN_F32, flags=0,
+          ws=FAKE, wsb=1 << 30):
+    return L.gdn_chunk_fwd(q, k, v, alpha, beta, S0, out, Sf, B, H, T, dk, dv, chunk, dtype,
+                           flags, ws, wsb, None)
+
+
+def test_argument_validation_before_launch(L):
+    assert _call(L, q=None) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, beta=None) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, out=None) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, k=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, Sf=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, B=-1) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, dtype=7) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, flags=8) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, dk=64, dv=128) == ops.GDN_ERR_INVALID_ARG
+    assert _call(L, dk=96, dv=96) == ops.GDN_ERR_UNSUPPORTED
+    assert _call(L, chunk=128) == ops.GDN_ERR_UNSUPPORTED
+    assert _call(L, chunk=0) == ops.GDN_ERR_UNSUPPORTED
+    assert _call(L, ws=None) == ops.GDN_ERR_WORKSPACE
+    assert _call(L, ws=FAKE + 16) == ops.GDN_ERR_WORKSPACE       # not 256-byte aligned
+    assert _call(L, wsb=1024) == ops.GDN_ERR_WORKSPACE           # too small
+    # empty batch: valid, nothing to do, no device access
+    assert _call(L, B=0) == ops.GDN_OK
+    assert _call(L, H=0) == ops.GDN_OK
+
+
+def test_deltaproduct_validation(L):
+    f = L.gdn_deltaproduct_fwd
+    args = [FAKE] * 5 + [None, FAKE, None]
+    assert f(*args, 1, 1, 8, 0, 64, 64, 64, ops.GDN_BF16, FAKE, 1 << 30, None) == ops.GDN_ERR_UNSUPPORTED
+    assert f(*args, 1, 1, 8, 5, 64, 64, 64, ops.GDN_BF16, FAKE, 1 << 30, None) == ops.GDN_ERR_UNSUPPORTED
+    bad = [None] + [FAKE] * 4 + [None, FAKE, None]
+    assert f(*bad, 1, 1, 8, 2, 64, 64, 64, ops.GDN_BF16, FAKE, 1 << 30, None) == ops.GDN_ERR_INVALID_ARG
+    assert f(*args, 1, 1, 8, 2, 64, 64, 64, ops.GDN_BF16, None, 0, None) == ops.GDN_ERR_WORKSPACE
+
+
+def test_status_query_needs_workspace(L):
+    assert L.gdn_workspace_status(None, None) == ops.GDN_ERR_WORKSPACE

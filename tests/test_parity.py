@@ -1,0 +1,146 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Small cases run the oracle on everything; the full-size configurations run
+the library exactly as bench.py does and compare sampled heads (the oracle
+handles (batch, head) pairs independently).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gated_delta_rule_fg_b200.inputs import CONFIGS, GdnConfig, make_inputs
+from _util import TOL_BF16, TOL_F32, parity, to_dev
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def _ops():
+    from gated_delta_rule_fg_b200 import ops
+    return ops
+
+
+def run_gdn(cfg, x, chunk=None):
+    ops = _ops()
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    out, sf = ops.chunk_fwd(to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt),
+                            to_dev(x["alpha"]), to_dev(x["beta"]), to_dev(x["S0"]),
+                            chunk=chunk or cfg.chunk, alpha_scalar=cfg.alpha_scalar,
+                            beta_scalar=cfg.beta_scalar)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), sf.cpu().numpy()
+
+
+def run_dp(cfg, x, chunk=None):
+    ops = _ops()
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    out, sf = ops.deltaproduct_fwd(to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt),
+                                   to_dev(x["gamma"]), to_dev(x["beta"]), to_dev(x["S0"]),
+                                   chunk=chunk or cfg.chunk)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), sf.cpu().numpy()
+
+
+def oracle_gdn(cfg, x, pairs=None):
+    return oracle.gdn_seq(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
+                          alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar, pairs=pairs)
+
+
+def oracle_dp(x, pairs=None):
+    return oracle.deltaproduct_seq(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["S0"], pairs=pairs)
+
+
+def check(cfg, got, ref, pairs=None):
+    tol = TOL_BF16 if cfg.dtype == "bf16" else TOL_F32
+    (o, s), (ro, rs) = got, ref
+    if pairs is not None:
+        idx_b = [b for b, _ in pairs]
+        idx_h = [h for _, h in pairs]
+        o, ro = o[idx_b, :, idx_h], ro[idx_b, :, idx_h]
+        s, rs = s[idx_b, idx_h], rs[idx_b, idx_h]
+    eo = parity(o, ro, tol, out_bf16=cfg.dtype == "bf16")
+    es = parity(s, rs, tol)
+    return eo, es
+
+
+# --------------------------------------------------------------------------- small, full oracle
+def test_config_fp32_small_exact_size():
+    """The float32 configuration at its stated size, every element."""
+    cfg = CONFIGS["fg2_f32_small"]
+    x = make_inputs(cfg)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+SMALL = []
+for dtype in ("f32", "bf16"):
+    for mode in ("fg2", "kda", "gdn", "deltanet"):
+        for T, chunk in ((1, 16), (15, 16), (64, 64), (250, 32), (250, 64), (131, 16)):
+            SMALL.append((dtype, mode, T, chunk))
+
+
+@pytest.mark.parametrize("dtype,mode,T,chunk", SMALL)
+def test_small_modes(dtype, mode, T, chunk):
+    """Every gate mode, ragged tails (T % chunk != 0), T < chunk and T = 1, both dtypes."""
+    cfg = GdnConfig("small", B=2, H=3, T=T, dk=64, dv=64, chunk=chunk, dtype=dtype,
+                    alpha_scalar=mode == "gdn", beta_scalar=mode in ("kda", "gdn", "deltanet"),
+                    s0_std=0.1 if T % 2 else 0.0, seed=T * 7 + chunk)
+    x = make_inputs(cfg)
+    if mode == "deltanet":
+        x["alpha"] = np.ones_like(x["alpha"])
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+@pytest.mark.parametrize("dk", [32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_head_dims(dk, dtype):
+    cfg = GdnConfig("dims", B=1, H=2, T=200, dk=dk, dv=dk, chunk=64 if dk == 128 else 32,
+                    dtype=dtype, s0_std=0.05, seed=dk)
+    x = make_inputs(cfg)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+def test_kda_unequal_head_dims():
+    """Scalar beta allows dk != dv."""
+    cfg = GdnConfig("kda_rect", B=1, H=2, T=100, dk=64, dv=128, chunk=32, beta_scalar=True,
+                    s0_std=0.05, seed=9)
+    x = make_inputs(cfg)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("nh,T,chunk", [(2, 40, 16), (2, 100, 64), (3, 33, 32), (1, 50, 16), (4, 17, 64)])
+def test_deltaproduct_small(dtype, nh, T, chunk):
+    cfg = GdnConfig("dp", B=2, H=2, T=T, dk=64, dv=64, chunk=chunk, dtype=dtype,
+                    deltaproduct_nh=nh, seed=nh * 100 + T)
+    x = make_inputs(cfg)
+    check(cfg, run_dp(cfg, x), oracle_dp(x))
+
+
+def test_strong_decay_small_alpha():
+    """Tiny alpha (log-decay span of hundreds inside a chunk) stays finite and exact."""
+    for dtype in ("f32", "bf16"):
+        cfg = GdnConfig("decay", B=1, H=2, T=130, dk=64, dv=64, chunk=64, dtype=dtype, seed=77)
+        x = make_inputs(cfg)
+        x["alpha"] = np.where(np.arange(130)[None, :, None, None] % 3 == 0, 1e-6,
+                              x["alpha"]).astype(np.float32)
+        check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+# --------------------------------------------------------------------------- full sizes, sampled
+FULL = ["kda_bf16", "fg2_prefill_32k", "fg2_train_b8", "deltaproduct_nh2"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_heads(name):
+    """Full-size configurations in the benchmark's launch configuration; the oracle
+    recomputes a sample of (batch, head) pairs, including the first and the last."""
+    cfg = CONFIGS[name]
+    x = make_inputs(cfg)
+    pairs = sorted({(0, 0), (cfg.B - 1, cfg.H - 1), (cfg.B // 2, cfg.H // 3)})
+    if cfg.deltaproduct_nh:
+        got = run_dp(cfg, x)
+        ref = oracle_dp(x, pairs=pairs)
+    else:
+        got = run_gdn(cfg, x)
+        ref = oracle_gdn(cfg, x, pairs=pairs)
+    check(cfg, got, ref, pairs=pairs)
