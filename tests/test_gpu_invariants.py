@@ -17,10 +17,13 @@ def _ops():
     return ops
 
 
-def _run(x, dtype, chunk, S0="x", **kw):
+_FROM_X = object()
+
+
+def _run(x, dtype, chunk, S0=_FROM_X, **kw):
     ops = _ops()
     dt = torch.bfloat16 if dtype == "bf16" else torch.float32
-    s0 = x["S0"] if S0 == "x" else S0
+    s0 = x["S0"] if S0 is _FROM_X else S0
     o, s = ops.chunk_fwd(to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt),
                          to_dev(x["alpha"]), to_dev(x["beta"]), to_dev(s0), chunk=chunk, **kw)
     torch.cuda.synchronize()
