@@ -144,3 +144,37 @@ def test_full_size_sampled_heads(name):
         got = run_gdn(cfg, x)
         ref = oracle_gdn(cfg, x, pairs=pairs)
     check(cfg, got, ref, pairs=pairs)
+
+
+# --------------------------------------------------------------------------- tensor-core path shapes
+TC = [(mode, T) for mode in ("fg2", "kda", "gdn", "deltanet") for T in (1, 63, 64, 65, 200)]
+
+
+@pytest.mark.parametrize("mode,T", TC)
+def test_tensor_core_shapes_modes(mode, T):
+    """bf16, chunk 64, dk = dv = 128 (the tensor-core kernels): every gate mode, T < chunk,
+    T = chunk, one past, ragged; nonzero S0 on odd T."""
+    cfg = GdnConfig("tc", B=2, H=2, T=T, dk=128, dv=128, chunk=64, dtype="bf16",
+                    alpha_scalar=mode == "gdn", beta_scalar=mode in ("kda", "gdn", "deltanet"),
+                    s0_std=0.1 if T % 2 else 0.0, seed=1000 + T)
+    x = make_inputs(cfg)
+    if mode == "deltanet":
+        x["alpha"] = np.ones_like(x["alpha"])
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+@pytest.mark.parametrize("nh,T", [(2, 100), (3, 70), (1, 130)])
+def test_tensor_core_deltaproduct(nh, T):
+    cfg = GdnConfig("tcdp", B=1, H=2, T=T, dk=128, dv=128, chunk=64, deltaproduct_nh=nh,
+                    s0_std=0.05, seed=2000 + T)
+    x = make_inputs(cfg)
+    check(cfg, run_dp(cfg, x), oracle_dp(x))
+
+
+def test_tensor_core_strong_decay_fallback():
+    """Chunks whose log-decay span is too wide for the factored fp16 Gram products take the
+    element-wise path; results stay exact."""
+    cfg = GdnConfig("tcdecay", B=1, H=2, T=200, dk=128, dv=128, chunk=64, seed=78)
+    x = make_inputs(cfg)
+    x["alpha"] = np.where(np.arange(200)[None, :, None, None] % 3 == 0, 1e-6, x["alpha"]).astype(np.float32)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
