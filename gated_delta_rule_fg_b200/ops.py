@@ -28,6 +28,8 @@ SIGNATURES = {
     "gdn_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                            ctypes.c_uint, _P, _SZ, _P]),
+    "gdn_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                   ctypes.c_uint, _P]),
     "gdn_deltaproduct_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_deltaproduct_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                   _I, _P, _SZ, _P]),
@@ -146,6 +148,30 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=False, be
                              _ptr(workspace), workspace.numel(), _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
+    return out, S_final
+
+
+def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=False,
+                      beta_scalar=False, out=None, S_final=None, want_state=True, stream=None):
+    """gdn_chunk_fwd_noalloc: as chunk_fwd, with the library's built-in 64 MiB scratch
+    instead of a caller workspace (for callers that cannot allocate device memory)."""
+    code = _dtype_code(q)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta"), (S0, "S0")):
+        _check(t, n, torch.float32)
+    flags = (GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = lib().gdn_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                     _ptr(out), _ptr(S_final), B, H, T, dk, dv, chunk, code, flags,
+                                     _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_noalloc")
     return out, S_final
 
 

@@ -103,6 +103,28 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
                            void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+/* gdn_chunk_fwd for callers that cannot allocate device memory (inside another
+ * framework's allocator or memory pool, in runtimes whose device memory is fixed
+ * at start-up, or while a stream is being captured): same arguments and result
+ * as gdn_chunk_fwd, without the workspace.  The paper has no counterpart; this
+ * is a deployment convenience of this library.
+ * The scratch is a 64 MiB array inside the library (a file-scope __device__
+ * array): every GPU on which the library's device code is loaded holds it until
+ * the process exits.  Sizes whose gdn_chunk_fwd_workspace_size exceeds 64 MiB
+ * (67108864 bytes) return GDN_ERR_WORKSPACE before anything is enqueued; other
+ * argument errors are reported as by gdn_chunk_fwd.  The first call on a device
+ * looks up the array's device address (with that device current) and caches it;
+ * make that first call before any stream capture.  All calls share the array
+ * and it keeps the last call's contents (its status word is cleared at the start
+ * of each call, device-side errors are not reported back); calls whose work can
+ * overlap on the GPU (different streams or threads) race on it. */
+gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta,
+                                   const float* S0, void* out, float* S_final,
+                                   int B, int H, int T, int dk, int dv, int chunk,
+                                   gdn_dtype_t dtype, unsigned flags,
+                                   cudaStream_t stream);
+
 /* Bytes of workspace gdn_deltaproduct_fwd needs (0 if invalid/unsupported). */
 size_t gdn_deltaproduct_fwd_workspace_size(int B, int H, int T, int n_h, int dk, int dv,
                                            int chunk, gdn_dtype_t dtype);
