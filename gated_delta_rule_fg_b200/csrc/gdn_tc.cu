@@ -35,13 +35,23 @@ constexpr int NS = 32;         // scan: columns per CTA
 constexpr int J = D / NS;      // scan: slices per head
 constexpr float kMaxHalfSpan = 6.0f;
 
-// Per (head, chunk) block in the workspace (bytes).
-constexpr uint32_t kOffAS1 = 0;          // [W; Qe] fp16 128x128, MN-major (mn=row, k=channel), SBO 2048, LBO 128
-constexpr uint32_t kOffAS2 = 32768;      // K'^T fp16 (mn=channel, k=row), MN-major, SBO 1024, LBO 128
-constexpr uint32_t kOffUp = 49152;       // U'  fp32 [J][C][NS]
-constexpr uint32_t kOffPUp = 81920;      // PU' fp32 [J][C][NS]
-constexpr uint32_t kOffGC = 114688;      // e^{g_last} fp32 [D]
+// Per (head, chunk) block in the workspace (bytes), written by the intra kernel and read
+// by the scan kernel.  "sw" rows: 32 fp16 per row, the four 16-byte groups of row x are
+// stored in the order g ^ ((x >> 1) & 3), so eight consecutive rows read as 16-byte
+// vectors hit eight different bank groups.
+constexpr uint32_t kOffN = 0;            // N = -K'^T W, fp16 128x128, K-major (m=i, k=c): SBO 2048, LBO 128
+constexpr uint32_t kOffQe = 32768;       // Qe fp16 64x128, MN-major (m=r, k=c): SBO 2048, LBO 128
+constexpr uint32_t kOffB = 49152;        // b = K'^T U', fp16 [J][128][NS] (sw rows)
+constexpr uint32_t kOffPU = 81920;       // PU', fp16 [J][64][NS] (sw rows)
+constexpr uint32_t kOffGC = 98304;       // e^{g_last}, fp32 [128]
+constexpr uint32_t kOffKp = 98816;       // K' fp16 (m=i, k=r), MN-major SBO 1024 LBO 128 (intra's own scratch)
 constexpr uint32_t kBlockBytes = 115200;
+// Fallback chunks (element-wise A and P) stage q^ (fp16) in the N area, k~ (fp16) in the
+// PU' area and g (fp32) in the b area; those areas are written only afterwards.
+
+__host__ __device__ __forceinline__ uint32_t sw_half(uint32_t row, uint32_t j) {
+    return row * NS + 8u * (((j >> 3) ^ ((row >> 1) & 3u))) + (j & 7u);
+}
 
 // intra shared memory map (bytes)
 constexpr uint32_t kR0 = 0;              // [KG; QG] fp16 K-major (row, ch): SBO 2048, LBO 128  -> later W~^T (K-major (ch, row): SBO 128, LBO 2048)
@@ -55,7 +65,8 @@ constexpr uint32_t kScr = 106496;        // 4 KB: per-warp log-decay totals, lat
 constexpr uint32_t kGref = 110592;       // g_ref [128]
 constexpr uint32_t kFK = 111104;         // e^{g_last - g_ref} [128]
 constexpr uint32_t kGlast = 111616;      // g_last [128]
-constexpr uint32_t kBar = 112128;        // mbarrier
+constexpr uint32_t kBar = 112128;        // mbarrier (MMA completion)
+constexpr uint32_t kBarK = 112144;       // mbarrier (K' reload)
 constexpr uint32_t kTmem = 112136;       // TMEM base address
 constexpr uint32_t kIntraSmem = 112192;
 
@@ -121,19 +132,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         tmem_alloc(tslot, kTmemCols);
         tmem_relinquish();
     }
+    uint64_t* bark = reinterpret_cast<uint64_t*>(sm + kBarK);
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bark, 1);
         fence_mbar_init();
     }
-    // identity operand (B layout: n = r, k = i)
-    for (int idx = tid; idx < 512; idx += NT) {
-        const int r = idx >> 3, j = idx & 7;
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = (8 * j + e == r) ? 1.f : 0.f;
-        st16(sm + kR5, off_kmajor(r, 8 * j, 1024, 128), f_to_h8(f));
-    }
-
     // ---------------------------------------------------------------- prep
     const int r = 8 * warp + (lane & 7);     // row of the chunk handled by this lane
     const int o0 = lane >> 3;                // channel octets o0, o0+4, o0+8, o0+12
@@ -147,13 +151,43 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(p.q);
     const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.k);
     const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.v);
+    const bool a_scalar = p.dp || p.alpha_scalar;
+    const bool b_scalar = p.dp || p.beta_scalar;
+    // beta (channel-wise) and v go to shared memory with register-free async copies: beta
+    // into a staging area over R3..R6 (free until the solve), v straight into its final
+    // place in R2 (converted in place later).  Everything is issued before any arithmetic.
+    float* bstage = reinterpret_cast<float*>(sm + kR3);
+    if (valid) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int o = o0 + 4 * j;
+            if (!b_scalar) {
+                float* dst = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+                cp_async16(dst, p.beta + rr.tok * D + 8 * o);
+                cp_async16(dst + 4, p.beta + rr.tok * D + 8 * o + 4);
+            }
+            cp_async16(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128), v + krow * D + 8 * o);
+        }
+    }
+    cp_async_commit();
     uint4 qp[4], kp[4];
-    float ssq = 0.f, ssk = 0.f;
+    float4 al0[4], al1[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
         qp[j] = (valid && rr.has_q) ? ldg16(q + rr.tok * D + 8 * o) : make_uint4(0, 0, 0, 0);
         kp[j] = valid ? ldg16(k + krow * D + 8 * o) : make_uint4(0, 0, 0, 0);
+        if (valid && !a_scalar) {
+            al0[j] = ldg16f(p.alpha + rr.tok * D + 8 * o);
+            al1[j] = ldg16f(p.alpha + rr.tok * D + 8 * o + 4);
+        } else {
+            al0[j] = make_float4(1.f, 1.f, 1.f, 1.f);
+            al1[j] = al0[j];
+        }
+    }
+    float ssq = 0.f, ssk = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
         float fq[8], fk[8];
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
@@ -170,8 +204,6 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     const float iq = rsqrtf(ssq + kNormEps);
     const float ik = rsqrtf(ssk + kNormEps);
 
-    const bool a_scalar = p.dp || p.alpha_scalar;
-    const bool b_scalar = p.dp || p.beta_scalar;
     float la_s = 0.f, b_s = 0.f;
     if (valid) {
         if (p.dp) {
@@ -191,8 +223,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) la[j][e] = valid ? la_s : 0.f;
         } else {
-            const float4 a0 = ldg16f(p.alpha + rr.tok * D + 8 * o);
-            const float4 a1 = ldg16f(p.alpha + rr.tok * D + 8 * o + 4);
+            const float4 a0 = al0[j], a1 = al1[j];
             la[j][0] = __logf(a0.x); la[j][1] = __logf(a0.y); la[j][2] = __logf(a0.z); la[j][3] = __logf(a0.w);
             la[j][4] = __logf(a1.x); la[j][5] = __logf(a1.y); la[j][6] = __logf(a1.z); la[j][7] = __logf(a1.w);
         }
@@ -232,9 +263,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     __syncthreads();
 
     // per octet: the fp16 operands
-    float* fb_g = reinterpret_cast<float*>(blk + kOffUp);                 // fallback scratch: g fp32 [C][D]
-    __half* fb_k = reinterpret_cast<__half*>(blk + kOffPUp);              // k~ fp16 [C][D]
-    __half* fb_q = reinterpret_cast<__half*>(blk + kOffPUp + C * D * 2);  // q^ fp16 [C][D]
+    float* fb_g = reinterpret_cast<float*>(blk + kOffB);                  // fallback scratch: g fp32 [C][D]
+    __half* fb_k = reinterpret_cast<__half*>(blk + kOffPU);               // k~ fp16 [C][D]
+    __half* fb_q = reinterpret_cast<__half*>(blk + kOffN);                // q^ fp16 [C][D]
+    cp_async_wait_all();     // this thread's own staged beta and v
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
@@ -246,12 +278,14 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) sb[e] = s;
         } else {
-            const float4 b0 = ldg16f(p.beta + rr.tok * D + 8 * o);
-            const float4 b1 = ldg16f(p.beta + rr.tok * D + 8 * o + 4);
+            const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+            const float4 b0 = *reinterpret_cast<const float4*>(bsrc);
+            const float4 b1 = *reinterpret_cast<const float4*>(bsrc + 4);
             sb[0] = sqrtf(b0.x); sb[1] = sqrtf(b0.y); sb[2] = sqrtf(b0.z); sb[3] = sqrtf(b0.w);
             sb[4] = sqrtf(b1.x); sb[5] = sqrtf(b1.y); sb[6] = sqrtf(b1.z); sb[7] = sqrtf(b1.w);
         }
-        const uint4 vp = valid ? ldg16(v + krow * D + 8 * o) : make_uint4(0, 0, 0, 0);
+        const uint4 vp = valid ? *reinterpret_cast<const uint4*>(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128))
+                               : make_uint4(0, 0, 0, 0);
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
         bf8_to_f(vp, fv);
@@ -279,7 +313,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         st16(sm + kR0, off_kmajor(64 + r, 8 * o, 2048, 128), f_to_h8(QG));
         st16(sm + kR1, off, f_to_h8(KIG));
         st16(sm + kR2, off, f_to_h8(VT));
-        *reinterpret_cast<uint4*>(blk + kOffAS2 + off_mnmajor(8 * o, r, 1024, 128)) = f_to_h8(KP);
+        *reinterpret_cast<uint4*>(blk + kOffKp + off_mnmajor(8 * o, r, 1024, 128)) = f_to_h8(KP);
         if (fallback) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) fb_g[r * D + 8 * o + e] = g[e];
@@ -288,12 +322,21 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         }
     }
     fence_async_smem();
+    asm volatile("fence.proxy.async.global;" ::: "memory");   // K' is read back by a bulk copy
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t t0 = *tslot;
     bool ok = true;
     uint32_t phase = 0;      // parity of the next completion of `bar`
+    // identity operand (B layout: n = r, k = i); its area held staged beta until now
+    for (int idx = tid; idx < 512; idx += NT) {
+        const int ri = idx >> 3, j = idx & 7;
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = (8 * j + e == ri) ? 1.f : 0.f;
+        st16(sm + kR5, off_kmajor(ri, 8 * j, 1024, 128), f_to_h8(f));
+    }
 
     // ---------------------------------------------------------------- A and P
     if (!fallback) {
@@ -369,60 +412,77 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     __syncthreads();
 
     // ---------------------------------------------------------------- T = (I + A)^{-1}
-    if (warp < 4 && lane < 16) {       // diagonal 16 x 16 blocks by forward substitution
-        const int bb = 16 * warp, jc = lane;
-        float t[16];
+    // Blocked forward substitution in fp32: four 16x16 diagonal blocks in registers
+    // (lane j carries column j; row r of A is broadcast by shuffles), then
+    // T10 = -T11 A10 T00 on 16x16 and 32x32 blocks.
+    if (warp < 4) {
+        const int bb = 16 * warp, jc = lane & 15;
+        float acol[16], t[16];
+#pragma unroll
+        for (int r2 = 0; r2 < 16; ++r2) acol[r2] = A32[sw64(bb + r2, bb + jc)];
 #pragma unroll
         for (int r2 = 0; r2 < 16; ++r2) {
             float acc = (r2 == jc) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (i >= jc && i < r2) acc -= A32[sw64(bb + r2, bb + i)] * t[i];
-            t[r2] = (r2 < jc) ? 0.f : acc;
+            for (int i = 0; i < r2; ++i) acc -= __shfl_sync(0xffffffffu, acol[r2], i) * t[i];
+            t[r2] = acc;
         }
+        if (lane < 16) {
 #pragma unroll
-        for (int r2 = 0; r2 < 16; ++r2) T32[sw64(bb + r2, bb + jc)] = t[r2];
+            for (int r2 = 0; r2 < 16; ++r2) T32[sw64(bb + r2, bb + jc)] = t[r2];
+        }
+    } else {
+        // zero the upper off-diagonal blocks the merges read: (0..15, 16..31), (32..47, 48..63)
+        const int u = tid - 128;
+        const int blk2 = u >> 6, e = (u & 63) * 4;
+        const int r0 = blk2 ? 32 : 0, c0 = blk2 ? 48 : 16;
+        *reinterpret_cast<float4*>(T32 + sw64(r0 + (e >> 4), c0 + (e & 15))) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    {   // 32 x 32 blocks: T10 = -T11 A10 T00 for the pairs (16..31 | 0..15) and (48..63 | 32..47)
+    {   // 16x16 merges for the block pairs (16..31 | 0..15) and (48..63 | 32..47)
         const int m = tid >> 7, qd = tid & 127;
-        const int rw = qd >> 3, jc = (qd & 7) * 2;
+        const int rw = qd >> 3, j2 = (qd & 7) * 2;
         const int base = 32 * m;
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int jj = jc + u;
-            float acc = 0.f;
-            for (int i = jj; i < 16; ++i) acc += A32[sw64(base + 16 + rw, base + i)] * T32[sw64(base + i, base + jj)];
-            scr[m * 256 + rw * 16 + jj] = acc;
+        for (int i = 0; i < 16; ++i) {
+            const float a = A32[sw64(base + 16 + rw, base + i)];
+            x0 = fmaf(a, T32[sw64(base + i, base + j2)], x0);
+            x1 = fmaf(a, T32[sw64(base + i, base + j2 + 1)], x1);
         }
+        scr[m * 256 + rw * 16 + j2] = x0;
+        scr[m * 256 + rw * 16 + j2 + 1] = x1;
         __syncthreads();
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int jj = jc + u;
-            float acc = 0.f;
-            for (int mm = 0; mm <= rw; ++mm) acc += T32[sw64(base + 16 + rw, base + 16 + mm)] * scr[m * 256 + mm * 16 + jj];
-            T32[sw64(base + 16 + rw, base + jj)] = -acc;
+        for (int mm = 0; mm < 16; ++mm) {
+            const float tt = T32[sw64(base + 16 + rw, base + 16 + mm)];
+            y0 = fmaf(tt, scr[m * 256 + mm * 16 + j2], y0);
+            y1 = fmaf(tt, scr[m * 256 + mm * 16 + j2 + 1], y1);
         }
+        T32[sw64(base + 16 + rw, base + j2)] = -y0;
+        T32[sw64(base + 16 + rw, base + j2 + 1)] = -y1;
     }
     __syncthreads();
-    {   // 64 x 64: T_BL = -T_BR A_BL T_TL (blocks of 32)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int idx = tid + NT * u;
-            const int rw = idx >> 5, jj = idx & 31;
-            float acc = 0.f;
-            for (int i = jj; i < 32; ++i) acc += A32[sw64(32 + rw, i)] * T32[sw64(i, jj)];
-            scr[rw * 32 + jj] = acc;
+    {   // 32x32 merge: T_BL = -T_BR (A_BL T_TL)
+        const int rw = tid >> 3, j4 = (tid & 7) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const float a = A32[sw64(32 + rw, i)];
+            const float4 tv = *reinterpret_cast<const float4*>(T32 + sw64(i, j4));
+            x.x = fmaf(a, tv.x, x.x); x.y = fmaf(a, tv.y, x.y); x.z = fmaf(a, tv.z, x.z); x.w = fmaf(a, tv.w, x.w);
         }
+        *reinterpret_cast<float4*>(scr + rw * 32 + j4) = x;
         __syncthreads();
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int idx = tid + NT * u;
-            const int rw = idx >> 5, jj = idx & 31;
-            float acc = 0.f;
-            for (int mm = 0; mm <= rw; ++mm) acc += T32[sw64(32 + rw, 32 + mm)] * scr[mm * 32 + jj];
-            T32[sw64(32 + rw, jj)] = -acc;
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int mm = 0; mm < 32; ++mm) {
+            const float tt = T32[sw64(32 + rw, 32 + mm)];
+            const float4 xv = *reinterpret_cast<const float4*>(scr + mm * 32 + j4);
+            y.x = fmaf(tt, xv.x, y.x); y.y = fmaf(tt, xv.y, y.y); y.z = fmaf(tt, xv.z, y.z); y.w = fmaf(tt, xv.w, y.w);
         }
+        *reinterpret_cast<float4*>(T32 + sw64(32 + rw, j4)) = make_float4(-y.x, -y.y, -y.z, -y.w);
     }
     __syncthreads();
     for (int idx = tid; idx < 512; idx += NT) {   // T -> fp16 B operand (n = r, k = i)
@@ -440,6 +500,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     __syncthreads();
     tc_fence_after();
 
+    // reload K' (written by the prep) into R1 as the A operand of the N and b products
+    if (ok && tid == 0) {
+        mbar_arrive_expect_tx(bark, 16384);
+        bulk_g2s(sm + kR1, blk + kOffKp, 16384, bark);
+    }
+
     // ---------------------------------------------------------------- W~^T = KG^T T^T ; U'^T = V~^T T^T
     if (ok) {
         if (tid == 0) {
@@ -454,53 +520,46 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     ok = __syncthreads_and(ok);
     if (!ok && tid == 0) record_timeout(p.status);
     tc_fence_after();
-    if (ok && warp < 4) {
-        const int ch = 32 * warp + lane;
-        const float er = __expf(gref[ch]);
-        const uint32_t lanebase = t0 + ((uint32_t)(32 * warp) << 16);
+    if (ok) {   // warps 0-3: W~^T -> R0 (K-major (c, r)); warps 4-7: U'^T -> R2 (K-major (j, r))
+        const int ch = 32 * (warp & 3) + lane;
+        const uint32_t lanebase = t0 + ((uint32_t)(32 * (warp & 3)) << 16);
+        const uint32_t col = warp < 4 ? 64 : 128;
+        uint8_t* dst = sm + (warp < 4 ? kR0 : kR2);
         float x0[32], x1[32];
-        tmem_ld32(lanebase + 64, x0);
-        tmem_ld32(lanebase + 96, x1);
+        tmem_ld32(lanebase + col, x0);
+        tmem_ld32(lanebase + col + 32, x1);
 #pragma unroll
-        for (int i0 = 0; i0 < C; i0 += 8) {
-            const float* src = (i0 < 32 ? x0 : x1) + (i0 & 31);
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = src[e] * er;
-            *reinterpret_cast<uint4*>(blk + kOffAS1 + off_mnmajor(i0, ch, 2048, 128)) = f_to_h8(f);
-            st16(sm + kR0, off_kmajor(ch, i0, 128, 2048), f_to_h8(src));
-        }
-        tmem_ld32(lanebase + 128, x0);
-        tmem_ld32(lanebase + 160, x1);
-        float* up = reinterpret_cast<float*>(blk + kOffUp) + (size_t)(ch / NS) * C * NS + (ch % NS);
-#pragma unroll
-        for (int i = 0; i < C; ++i) up[i * NS] = i < 32 ? x0[i] : x1[i - 32];
-#pragma unroll
-        for (int i0 = 0; i0 < C; i0 += 8) st16(sm + kR2, off_kmajor(ch, i0, 128, 2048), f_to_h8((i0 < 32 ? x0 : x1) + (i0 & 31)));
+        for (int i0 = 0; i0 < C; i0 += 8) st16(dst, off_kmajor(ch, i0, 128, 2048), f_to_h8((i0 < 32 ? x0 : x1) + (i0 & 31)));
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
-    // ---------------------------------------------------------------- (Qe e^{-g_ref})^T and PU'^T
+    // ---------------------------------------------------------------- (Qe e^{-g_ref})^T, PU'^T, N~ = -K'^T W~
     if (ok) {
+        const bool kok = mbar_wait(bark, 0);
         if (tid == 0) {
-            mma_f16_k(t0 + 0, smem_u32(sm + kR0), 2048, 128, smem_u32(sm + kR4), 128, 1024,
-                      idesc_f16(128, 64, false, false, true), C, false);
-            mma_f16_k(t0 + 0, smem_u32(sm + kR0 + 16384), 2048, 128, smem_u32(sm + kR5), 128, 1024,
-                      idesc_f16(128, 64, true, false), C, true);
-            mma_f16_k(t0 + 192, smem_u32(sm + kR2), 2048, 128, smem_u32(sm + kR4), 128, 1024,
-                      idesc_f16(128, 64, false, false), C, false);
-            mma_commit(bar);
+            if (kok) {
+                tc_fence_after();
+                mma_f16_k(t0 + 0, smem_u32(sm + kR0), 2048, 128, smem_u32(sm + kR4), 128, 1024,
+                          idesc_f16(128, 64, false, false, true), C, false);
+                mma_f16_k(t0 + 0, smem_u32(sm + kR0 + 16384), 2048, 128, smem_u32(sm + kR5), 128, 1024,
+                          idesc_f16(128, 64, true, false), C, true);
+                mma_f16_k(t0 + 192, smem_u32(sm + kR2), 2048, 128, smem_u32(sm + kR4), 128, 1024,
+                          idesc_f16(128, 64, false, false), C, false);
+                mma_f16_k(t0 + 64, smem_u32(sm + kR1), 128, 1024, smem_u32(sm + kR0), 2048, 128,
+                          idesc_f16(128, 128, true, false, true), C, false);
+                mma_commit(bar);
+            }
         }
-        ok = mbar_wait(bar, phase);
+        ok = kok && mbar_wait(bar, phase);
         phase ^= 1u;
     }
     ok = __syncthreads_and(ok);
     if (!ok && tid == 0) record_timeout(p.status);
     tc_fence_after();
-    if (ok && warp < 4) {
+    if (ok && warp < 4) {        // Qe -> block (MN-major (r, c)); PU' -> block (fp16, sw rows)
         const int ch = 32 * warp + lane;
         const float er = __expf(gref[ch]);
         const uint32_t lanebase = t0 + ((uint32_t)(32 * warp) << 16);
@@ -513,13 +572,58 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             float f[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = src[e] * er;
-            *reinterpret_cast<uint4*>(blk + kOffAS1 + off_mnmajor(64 + r0, ch, 2048, 128)) = f_to_h8(f);
+            *reinterpret_cast<uint4*>(blk + kOffQe + off_mnmajor(r0, ch, 2048, 128)) = f_to_h8(f);
         }
         tmem_ld32(lanebase + 192, x0);
         tmem_ld32(lanebase + 224, x1);
-        float* pu = reinterpret_cast<float*>(blk + kOffPUp) + (size_t)(ch / NS) * C * NS + (ch % NS);
+        __half* pu = reinterpret_cast<__half*>(blk + kOffPU) + (size_t)(ch / NS) * C * NS;
 #pragma unroll
-        for (int i = 0; i < C; ++i) pu[i * NS] = i < 32 ? x0[i] : x1[i - 32];
+        for (int r2 = 0; r2 < C; ++r2) pu[sw_half(r2, ch % NS)] = __float2half_rn(r2 < 32 ? x0[r2] : x1[r2 - 32]);
+    } else if (ok) {             // N = N~ * e^{g_ref[c]} (column scale) -> block (K-major (i, c))
+        const int row = 32 * (warp & 3) + lane;
+        const uint32_t lanebase = t0 + ((uint32_t)(32 * (warp & 3)) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            float x[32];
+            tmem_ld32(lanebase + 64 + c0, x);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= __expf(gref[c0 + e]);
+#pragma unroll
+            for (int g8 = 0; g8 < 32; g8 += 8)
+                *reinterpret_cast<uint4*>(blk + kOffN + off_kmajor(row, c0 + g8, 2048, 128)) = f_to_h8(x + g8);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---------------------------------------------------------------- b = K'^T U'
+    if (ok) {
+        if (tid == 0) {
+            mma_f16_k(t0 + 0, smem_u32(sm + kR1), 128, 1024, smem_u32(sm + kR2), 2048, 128,
+                      idesc_f16(128, 128, true, false), C, false);
+            mma_commit(bar);
+        }
+        ok = mbar_wait(bar, phase);
+        phase ^= 1u;
+    }
+    ok = __syncthreads_and(ok);
+    if (!ok && tid == 0) record_timeout(p.status);
+    tc_fence_after();
+    if (ok) {                    // warps 0-3: columns 0-63, warps 4-7: columns 64-127
+        const int row = 32 * (warp & 3) + lane;
+        const uint32_t lanebase = t0 + ((uint32_t)(32 * (warp & 3)) << 16);
+        const int cbase = warp < 4 ? 0 : 64;
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+            float x[32];
+            tmem_ld32(lanebase + cbase + c0, x);
+            const int j0 = cbase + c0;                  // one full 32-column slice
+            __half* bb = reinterpret_cast<__half*>(blk + kOffB) + (size_t)(j0 / NS) * D * NS;
+#pragma unroll
+            for (int g8 = 0; g8 < 32; g8 += 8)
+                *reinterpret_cast<uint4*>(bb + sw_half(row, g8)) = f_to_h8(x + g8);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -527,16 +631,32 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 }
 
 // ============================================================================ scan
-constexpr int kScanThreads = 160;              // 4 epilogue warps + 1 producer warp
-constexpr uint32_t kStageBytes = 32768 + 16384 + 8192 + 8192 + 512;   // AS1, AS2, U', PU', gC
-constexpr uint32_t kSAS1 = 0, kSAS2 = 32768, kSUp = 49152, kSPUp = 57344, kSGC = 65536;
-constexpr uint32_t kStage0 = 0;
-constexpr uint32_t kStageStride = 66560;       // kStageBytes rounded up to 1 KB
-constexpr uint32_t kSop = 2 * kStageStride;    // S fp16 B operand (k = ch, n = j): MN-major SBO 2048 LBO 128 (8 KB)
-constexpr uint32_t kUop = kSop + 8192;         // U fp16 B operand (k = r, n = j): MN-major SBO 1024 LBO 128 (4 KB)
-constexpr uint32_t kSBar = kUop + 4096;        // full[2], empty[2], s1, s2
-constexpr uint32_t kSTmem = kSBar + 64;
-constexpr uint32_t kScanSmem = kSTmem + 64;
+// One CTA per (head, 32-column slice).  Per chunk c, with S_c in fp32 registers (row i
+// per thread) and its fp16 copy in Sop[c % 3]:
+//   MMA_S: D_S = N_c S_c          -> S_{c+1} = Diag(gC) S_c + D_S + b_c   (the serial chain)
+//   MMA_O: D_O[c & 1] = Qe_c S_c  -> O_c = D_O + PU'_c                     (off the chain)
+// MMA_O(c) is issued right after MMA_S(c+1), so it runs in the tensor pipe while the state
+// epilogue of chunk c+1 works instead of sitting in front of the next chain MMA; the fp16
+// state therefore keeps three buffers.
+// Roles: warps 0-3 carry the state (one d_k row per thread), warps 4-7 form the outputs
+// (the M = 64 accumulator puts row r in lane (r%16) + 32*(r/16)), warp 8 streams the
+// per-chunk blocks with bulk copies into two rings ({N, b slice, gC} x 3 and
+// {Qe, PU' slice} x 4), and one thread of warp 9 issues every MMA.  All hand-offs are
+// mbarriers with bounded waits.
+constexpr int kScanThreads = 320;
+constexpr int kNB = 3, kQP = 4;
+constexpr uint32_t kNBBytes = 32768 + 8192 + 512;
+constexpr uint32_t kNBStride = 41472;
+constexpr uint32_t kQPBytes = 16384 + 4096;
+constexpr uint32_t kQPStride = 20480;
+constexpr uint32_t kSN = 0, kSB = 32768, kSG = 40960;      // within an NB stage
+constexpr uint32_t kSQe = 0, kSPU = 16384;                 // within a QP stage
+constexpr uint32_t kRingNB = 0;
+constexpr uint32_t kRingQP = kRingNB + kNB * kNBStride;    // 124416
+constexpr uint32_t kSop = kRingQP + kQP * kQPStride;       // 206336: 3 x 8 KB, S fp16 (k = i, n = j) MN-major SBO 2048 LBO 128
+constexpr uint32_t kSBar = kSop + 3 * 8192;                // 230912: mbarriers
+constexpr uint32_t kSTmem = kSBar + 256;
+constexpr uint32_t kScanSmem = kSTmem + 64;                // 231232
 
 __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -544,131 +664,140 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kSBar);
-    uint64_t* empty = full + 2;
-    uint64_t* s1 = full + 4;
-    uint64_t* s2 = full + 5;
+    uint64_t* fullNB = reinterpret_cast<uint64_t*>(sm + kSBar);
+    uint64_t* emptyNB = fullNB + kNB;
+    uint64_t* fullQP = emptyNB + kNB;
+    uint64_t* emptyQP = fullQP + kQP;
+    uint64_t* bar_s = emptyQP + kQP;       // MMA_S done
+    uint64_t* bar_o = bar_s + 1;           // [2] MMA_O done, per D_O buffer
+    uint64_t* s_ready = bar_o + 2;         // S_c written to Sop (4 warp arrivals)
+    uint64_t* o_free = s_ready + 1;        // [2] D_O buffer read (4 warp arrivals)
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kSTmem);
     const uint8_t* blocks = static_cast<const uint8_t*>(p.inter) + (size_t)bh * p.NC * kBlockBytes;
 
     if (warp == 0) {
-        tmem_alloc(tslot, 64);
+        tmem_alloc(tslot, 128);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(&empty[0], 1);
-        mbar_init(&empty[1], 1);
-        mbar_init(s1, 1);
-        mbar_init(s2, 1);
+        for (int i = 0; i < kNB; ++i) { mbar_init(&fullNB[i], 1); mbar_init(&emptyNB[i], 4); }
+        for (int i = 0; i < kQP; ++i) { mbar_init(&fullQP[i], 1); mbar_init(&emptyQP[i], 4); }
+        mbar_init(bar_s, 1);
+        mbar_init(&bar_o[0], 1);
+        mbar_init(&bar_o[1], 1);
+        mbar_init(s_ready, 4);
+        mbar_init(&o_free[0], 4);
+        mbar_init(&o_free[1], 4);
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t t0 = *tslot;
+    const uint32_t tS = t0, tO = t0 + 32;                  // D_S (32 columns); D_O[0], D_O[1]
+    bool ok = true;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int ch = 0; ch < p.NC; ++ch) {
-                const int st = ch & 1;
-                if (ch >= 2 && !mbar_wait(&empty[st], ((ch >> 1) - 1) & 1)) {
-                    record_timeout(p.status);
-                    break;
-                }
-                uint8_t* dst = sm + kStage0 + st * kStageStride;
+            for (int ch = 0; ch < p.NC && ok; ++ch) {
                 const uint8_t* src = blocks + (size_t)ch * kBlockBytes;
-                mbar_arrive_expect_tx(&full[st], kStageBytes);
-                bulk_g2s(dst + kSAS1, src + kOffAS1, 32768, &full[st]);
-                bulk_g2s(dst + kSAS2, src + kOffAS2, 16384, &full[st]);
-                bulk_g2s(dst + kSUp, src + kOffUp + (size_t)slice * C * NS * 4, 8192, &full[st]);
-                bulk_g2s(dst + kSPUp, src + kOffPUp + (size_t)slice * C * NS * 4, 8192, &full[st]);
-                bulk_g2s(dst + kSGC, src + kOffGC, 512, &full[st]);
+                const int s3 = ch % kNB, s4 = ch % kQP;
+                if (ch >= kNB && !mbar_wait(&emptyNB[s3], ((ch / kNB) - 1) & 1)) { ok = false; break; }
+                uint8_t* d3 = sm + kRingNB + s3 * kNBStride;
+                mbar_arrive_expect_tx(&fullNB[s3], kNBBytes);
+                bulk_g2s(d3 + kSN, src + kOffN, 32768, &fullNB[s3]);
+                bulk_g2s(d3 + kSB, src + kOffB + (size_t)slice * D * NS * 2, 8192, &fullNB[s3]);
+                bulk_g2s(d3 + kSG, src + kOffGC, 512, &fullNB[s3]);
+                if (ch >= kQP && !mbar_wait(&emptyQP[s4], ((ch / kQP) - 1) & 1)) { ok = false; break; }
+                uint8_t* d4 = sm + kRingQP + s4 * kQPStride;
+                mbar_arrive_expect_tx(&fullQP[s4], kQPBytes);
+                bulk_g2s(d4 + kSQe, src + kOffQe, 16384, &fullQP[s4]);
+                bulk_g2s(d4 + kSPU, src + kOffPU + (size_t)slice * C * NS * 2, 4096, &fullQP[s4]);
             }
+            if (!ok) record_timeout(p.status);
         }
-    } else {
-        // ------------------------------------------------------------ state chain (128 threads)
-        const int row = tid;                           // TMEM lane: d_k row of S / chunk row of D1
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ MMA issuer (one thread)
+        if (lane == 0) {
+            const uint32_t idS = idesc_f16(128, NS, false, true);
+            const uint32_t idO = idesc_f16(64, NS, true, true);
+            // MMA_O of chunk cc (reads Sop[cc % 3] and the QP stage of cc)
+            auto issue_o = [&](int cc) -> bool {
+                const int s4 = cc % kQP;
+                if (cc >= 2 && !mbar_wait(&o_free[cc & 1], ((cc >> 1) - 1) & 1)) return false;
+                if (!mbar_wait(&fullQP[s4], (cc / kQP) & 1)) return false;
+                tc_fence_after();
+                const uint64_t a0 = sdesc(smem_u32(sm + kRingQP + s4 * kQPStride + kSQe), 128, 2048);
+                const uint64_t b0 = sdesc(smem_u32(sm + kSop + (cc % 3) * 8192), 128, 2048);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) mma_f16(tO + 32 * (cc & 1), a0 + 16 * kk, b0 + 16 * kk, idO, kk > 0);
+                mma_commit(&bar_o[cc & 1]);
+                return true;
+            };
+            for (int ch = 0; ch < p.NC && ok; ++ch) {
+                const int s3 = ch % kNB;
+                if (!mbar_wait(s_ready, ch & 1) || !mbar_wait(&fullNB[s3], (ch / kNB) & 1)) { ok = false; break; }
+                tc_fence_after();
+                {
+                    const uint64_t a0 = sdesc(smem_u32(sm + kRingNB + s3 * kNBStride + kSN), 128, 2048);
+                    const uint64_t b0 = sdesc(smem_u32(sm + kSop + (ch % 3) * 8192), 128, 2048);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) mma_f16(tS, a0 + 16 * kk, b0 + 16 * kk, idS, kk > 0);
+                    mma_commit(bar_s);
+                }
+                if (ch > 0 && !issue_o(ch - 1)) { ok = false; break; }
+            }
+            if (ok && p.NC > 0) ok = issue_o(p.NC - 1);
+            if (!ok) record_timeout(p.status);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ state chain
+        const int row = tid;                                   // d_k row of S (TMEM lane)
         const int j0 = slice * NS;
-        const uint32_t lanebase = t0 + ((uint32_t)(32 * warp) << 16);
+        const uint32_t lanebase = (uint32_t)(32 * warp) << 16;
         float S[NS];
 #pragma unroll
         for (int j = 0; j < NS; ++j) S[j] = p.S0 ? p.S0[((size_t)bh * D + row) * D + j0 + j] : 0.f;
 #pragma unroll
         for (int j = 0; j < NS; j += 8) st16(sm + kSop, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
         fence_async_smem();
-        named_barrier(1, 128);
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-        const uint32_t id1 = idesc_f16(128, NS, true, true);
-        const uint32_t id2 = idesc_f16(128, NS, true, true);
-        bool ok = true;
-        for (int ch = 0; ch < p.NC; ++ch) {
-            const int st = ch & 1;
-            uint8_t* stg = sm + kStage0 + st * kStageStride;
-            bool mine = mbar_wait(&full[st], (ch >> 1) & 1);
-            if (tid == 0 && mine) {
-                tc_fence_after();
-                mma_f16_k(t0 + 0, smem_u32(stg + kSAS1), 128, 2048, smem_u32(sm + kSop), 128, 2048, id1, D, false);
-                mma_commit(s1);
-            }
-            mine = mine && mbar_wait(s1, ch & 1);
-            tc_fence_after();
-            float d[NS];
-            if (mine) {
-                tmem_ld32(lanebase + 0, d);
-                const float* up = reinterpret_cast<const float*>(stg + kSUp);
-                const float* pu = reinterpret_cast<const float*>(stg + kSPUp);
-                if (row < C) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_ready);
+        for (int ch = 0; ch < p.NC && ok; ++ch) {
+            const int s3 = ch % kNB;
+            const uint8_t* nb = sm + kRingNB + s3 * kNBStride;
+            if (!__all_sync(0xffffffffu, mbar_wait(&fullNB[s3], (ch / kNB) & 1))) { ok = false; break; }
+            const __half* bsm = reinterpret_cast<const __half*>(nb + kSB);
+            float bv[NS];
 #pragma unroll
-                    for (int j = 0; j < NS; ++j) d[j] = up[row * NS + j] - d[j];
+            for (int g8 = 0; g8 < NS; g8 += 8) {
+                const uint4 v = *reinterpret_cast<const uint4*>(bsm + sw_half(row, g8));
+                const __half2* hh = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
-                    for (int j = 0; j < NS; j += 8) st16(sm + kUop, off_mnmajor(j, row, 1024, 128), f_to_h8(d + j));
-                    fence_async_smem();
-                } else {
-                    const int rw = row - C;
-                    const int s = ch * C + rw;
-                    if (s < p.L) {
-                        const RowRef ro = row_ref(p, b, h, s);
-                        if (ro.has_q) {
-                            uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + j0);
-#pragma unroll
-                            for (int j = 0; j < NS; j += 8) {
-                                __nv_bfloat162 o2[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    o2[e] = __floats2bfloat162_rn(pu[rw * NS + j + 2 * e] + d[j + 2 * e],
-                                                                  pu[rw * NS + j + 2 * e + 1] + d[j + 2 * e + 1]);
-                                dst[j / 8] = *reinterpret_cast<uint4*>(o2);
-                            }
-                        }
-                    }
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(hh[e]);
+                    bv[g8 + 2 * e] = f.x;
+                    bv[g8 + 2 * e + 1] = f.y;
                 }
             }
-            tc_fence_before();
-            ok = named_barrier_and(1, 128, mine);
-            if (!ok) break;
-            if (tid == 0) {
-                tc_fence_after();
-                mma_f16_k(t0 + 32, smem_u32(stg + kSAS2), 128, 1024, smem_u32(sm + kUop), 128, 1024, id2, C, false);
-                mma_commit(s2);
-            }
-            mine = mbar_wait(s2, ch & 1);
+            const float gc = reinterpret_cast<const float*>(nb + kSG)[row];
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_s, ch & 1))) { ok = false; break; }
             tc_fence_after();
-            if (mine) {
-                tmem_ld32(lanebase + 32, d);
-                const float gc = reinterpret_cast<const float*>(stg + kSGC)[row];
+            float d[NS];
+            tmem_ld32(t0 + lanebase + (tS - t0), d);
 #pragma unroll
-                for (int j = 0; j < NS; ++j) S[j] = gc * S[j] + d[j];
+            for (int j = 0; j < NS; ++j) S[j] = fmaf(gc, S[j], d[j] + bv[j]);
+            uint8_t* snext = sm + kSop + ((ch + 1) % 3) * 8192;
 #pragma unroll
-                for (int j = 0; j < NS; j += 8) st16(sm + kSop, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
-                fence_async_smem();
-            }
+            for (int j = 0; j < NS; j += 8) st16(snext, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
+            fence_async_smem();
             tc_fence_before();
-            ok = named_barrier_and(1, 128, mine);
-            if (!ok) break;
-            if (tid == 0) mbar_arrive(&empty[st]);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(s_ready);                          // S_{ch+1} is in Sop[(ch+1) % 3]
+                mbar_arrive(&emptyNB[s3]);
+            }
         }
         if (!ok) {
             if (lane == 0) record_timeout(p.status);
@@ -677,10 +806,56 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
 #pragma unroll
             for (int j = 0; j < NS; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
+    } else {
+        // ------------------------------------------------------------ outputs (warps 4-7)
+        const int wq = warp - 4;                               // TMEM lane quarter
+        const int j0 = slice * NS;
+        const uint32_t lanebase = (uint32_t)(32 * wq) << 16;
+        const int rw = 16 * wq + lane;                         // output row (valid for lane < 16)
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+        for (int ch = 0; ch < p.NC && ok; ++ch) {
+            const int s4 = ch % kQP;
+            const bool got = mbar_wait(&fullQP[s4], (ch / kQP) & 1) && mbar_wait(&bar_o[ch & 1], (ch >> 1) & 1);
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float d[NS];
+            tmem_ld32(t0 + lanebase + (tO - t0) + 32 * (ch & 1), d);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[ch & 1]);
+            if (lane < 16) {
+                const int s = ch * C + rw;
+                if (s < p.L) {
+                    const RowRef ro = row_ref(p, b, h, s);
+                    if (ro.has_q) {
+                        const __half* pu = reinterpret_cast<const __half*>(sm + kRingQP + s4 * kQPStride + kSPU);
+                        uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + j0);
+#pragma unroll
+                        for (int g8 = 0; g8 < NS; g8 += 8) {
+                            const uint4 pv = *reinterpret_cast<const uint4*>(pu + sw_half(rw, g8));
+                            const __half2* ph = reinterpret_cast<const __half2*>(&pv);
+                            __nv_bfloat162 o2[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 pf = __half22float2(ph[e]);
+                                o2[e] = __floats2bfloat162_rn(pf.x + d[g8 + 2 * e], pf.y + d[g8 + 2 * e + 1]);
+                            }
+                            dst[g8 / 8] = *reinterpret_cast<uint4*>(o2);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&emptyQP[s4]);
+        }
+        if (!ok && lane == 0) record_timeout(p.status);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(t0, 64);
+    if (warp == 0) tmem_dealloc(t0, 128);
 }
 
 }  // namespace tc

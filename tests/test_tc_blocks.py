@@ -1,5 +1,5 @@
 """Unit check of the tensor-core intra-chunk kernel: decode the per-chunk blocks it
-writes into the workspace (W, Qe, K', U', PU', e^{g_last}) and compare them with the
+writes into the workspace (N = -K'^T W, Qe, K', b = K'^T U', PU', e^{g_last}) and compare them with the
 same quantities formed in fp64 numpy from their definitions (chunk-local cumulative
 log-decay g, A and P with the decay taken element by element, T = (I + A)^{-1}).
 The block layout is the library's internal contract between its two kernels."""
@@ -14,25 +14,37 @@ torch = pytest.importorskip("torch")
 
 C, D, NS = 64, 128, 32
 BLOCK = 115200
-OFF_AS1, OFF_AS2, OFF_UP, OFF_PUP, OFF_GC = 0, 32768, 49152, 81920, 114688
+OFF_N, OFF_QE, OFF_B, OFF_PU, OFF_GC, OFF_KP = 0, 32768, 49152, 81920, 98304, 98816
 
 
 def off_mn(mn, k, sbo, lbo):
     return (mn % 8) * 2 + (k % 8) * 16 + (mn // 8) * sbo + (k // 8) * lbo
 
 
+def off_k(mn, k, sbo, lbo):
+    return (mn % 8) * 16 + (k % 8) * 2 + (mn // 8) * sbo + (k // 8) * lbo
+
+
+def sw(row, j):
+    return row * NS + 8 * ((j // 8) ^ ((row // 2) % 4)) + j % 8
+
+
 def decode(blk):
     h = blk.view(np.float16)
     f = blk.view(np.float32)
-    rows, chs = np.meshgrid(np.arange(128), np.arange(128), indexing="ij")
-    AS1 = h[(OFF_AS1 + off_mn(rows, chs, 2048, 128)) // 2].astype(np.float64)
-    W, Qe = AS1[:64], AS1[64:]
-    ch2, r2 = np.meshgrid(np.arange(128), np.arange(64), indexing="ij")
-    Kp = h[(OFF_AS2 + off_mn(ch2, r2, 1024, 128)) // 2].astype(np.float64).T      # [r][ch]
-    Up = f[OFF_UP // 4:OFF_UP // 4 + C * D].reshape(D // NS, C, NS).transpose(1, 0, 2).reshape(C, D)
-    PUp = f[OFF_PUP // 4:OFF_PUP // 4 + C * D].reshape(D // NS, C, NS).transpose(1, 0, 2).reshape(C, D)
+    i2, c2 = np.meshgrid(np.arange(128), np.arange(128), indexing="ij")
+    N = h[(OFF_N + off_k(i2, c2, 2048, 128)) // 2].astype(np.float64)
+    r2, c3 = np.meshgrid(np.arange(64), np.arange(128), indexing="ij")
+    Qe = h[(OFF_QE + off_mn(r2, c3, 2048, 128)) // 2].astype(np.float64)
+    ch2, rr2 = np.meshgrid(np.arange(128), np.arange(64), indexing="ij")
+    Kp = h[(OFF_KP + off_mn(ch2, rr2, 1024, 128)) // 2].astype(np.float64).T       # [r][ch]
+    jj = np.arange(128)
+    bi, bj = np.meshgrid(np.arange(128), jj, indexing="ij")
+    b = h[OFF_B // 2 + (bj // NS) * 128 * NS + sw(bi, bj % NS)].astype(np.float64)
+    pr, pj = np.meshgrid(np.arange(64), jj, indexing="ij")
+    PU = h[OFF_PU // 2 + (pj // NS) * 64 * NS + sw(pr, pj % NS)].astype(np.float64)
     gC = f[OFF_GC // 4:OFF_GC // 4 + D]
-    return dict(W=W, Qe=Qe, Kp=Kp, Up=Up.astype(np.float64), PUp=PUp.astype(np.float64), gC=gC)
+    return dict(N=N, Qe=Qe, Kp=Kp, b=b, PUp=PU, gC=gC)
 
 
 def expected(x, h, c0, n, beta_scalar=False):
@@ -57,8 +69,8 @@ def expected(x, h, c0, n, beta_scalar=False):
     T = np.linalg.inv(np.eye(C) + A)
     W = T @ (kt * np.exp(g))
     Up = T @ vt
-    return dict(W=W, Qe=qh * np.exp(g) - P @ W, Kp=kt * np.exp(g[-1] - g), Up=Up, PUp=P @ Up,
-                gC=np.exp(g[-1]))
+    Kp = kt * np.exp(g[-1] - g)
+    return dict(N=-Kp.T @ W, Qe=qh * np.exp(g) - P @ W, Kp=Kp, b=Kp.T @ Up, PUp=P @ Up, gC=np.exp(g[-1]))
 
 
 def _rel(a, b):
@@ -86,5 +98,5 @@ def test_intra_blocks(alpha_mode):
             n = min(C, T - c * C)
             got = decode(raw[(h * NC + c) * BLOCK:(h * NC + c + 1) * BLOCK])
             want = expected(x, h, c * C, n)
-            for key, tol in (("W", 3e-3), ("Qe", 3e-3), ("Kp", 2e-3), ("Up", 3e-3), ("PUp", 3e-3), ("gC", 1e-5)):
+            for key, tol in (("N", 3e-3), ("Qe", 3e-3), ("Kp", 2e-3), ("b", 3e-3), ("PUp", 3e-3), ("gC", 1e-5)):
                 assert _rel(got[key], want[key]) < tol, (h, c, key, _rel(got[key], want[key]))
