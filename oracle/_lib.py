@@ -34,7 +34,7 @@ def lib():
         _lib = ctypes.CDLL(build())
         f = ctypes.c_void_p
         i = ctypes.c_int
-        _lib.oracle_gdn_seq.argtypes = [f, f, f, f, f, f, f, f, i, i, i, i, i, i, i,
+        _lib.oracle_gdn_seq.argtypes = [f, f, f, f, f, f, f, f, f, i, i, i, i, i, i, i,
                                         ctypes.c_double, f, i, i]
         _lib.oracle_gdn_seq.restype = i
         _lib.oracle_deltaproduct_seq.argtypes = [f, f, f, f, f, f, f, f, i, i, i, i, i, i,
@@ -64,26 +64,28 @@ def max_threads() -> int:
 
 
 def gdn_seq(q, k, v, alpha, beta, S0=None, *, alpha_scalar=False, beta_scalar=False,
-            eps=1e-6, pairs=None, nthreads=0):
+            eps=1e-6, pairs=None, nthreads=0, beta_v=None):
     """Token-by-token FG^2-GDN recurrence in fp64.
 
     q, k: [B,T,H,dk]; v: [B,T,H,dv]; alpha, beta: [B,T,H,dk] or [B,T,H] when
-    scalar; S0: [B,H,dk,dv] or None (zero state).  Inputs are read as float32
+    scalar; S0: [B,H,dk,dv] or None (zero state).  beta_v ([B,T,H,dv], or [B,T,H]
+    when scalar) selects FG^2-GDN+: beta then scales the keys and beta_v the values.
+    Inputs are read as float32
     values (bf16 data must be passed exactly upcast).  Returns (o, S_final) in
     float64, o [B,T,H,dv], S_final [B,H,dk,dv].  With `pairs` (a list of
     (b, h)), only those heads are computed and the other entries stay zero.
     """
-    q, k, v, alpha, beta, S0 = map(_f32, (q, k, v, alpha, beta, S0))
+    q, k, v, alpha, beta, beta_v, S0 = map(_f32, (q, k, v, alpha, beta, beta_v, S0))
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, T, H, dv), dtype=np.float64)
     sf = np.zeros((B, H, dk, dv), dtype=np.float64)
     parr, npairs = _pairs(pairs)
-    rc = lib().oracle_gdn_seq(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+    rc = lib().oracle_gdn_seq(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(beta_v), _ptr(S0),
                               _ptr(o), _ptr(sf), B, H, T, dk, dv, int(alpha_scalar),
                               int(beta_scalar), float(eps), _ptr(parr), npairs, int(nthreads))
     if rc != 0:
-        raise ValueError("channel-wise beta needs dk == dv")
+        raise ValueError("channel-wise beta needs dk == dv (or a separate beta_v)")
     return o, sf
 
 

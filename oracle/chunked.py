@@ -31,17 +31,20 @@ def _normalise(x, eps):
 
 
 def gdn_chunked(q, k, v, alpha, beta, S0=None, *, chunk, alpha_scalar=False,
-                beta_scalar=False, eps=1e-6):
+                beta_scalar=False, eps=1e-6, beta_v=None):
     """Chunkwise evaluation of the recurrence; same arguments and returns as
-    oracle.gdn_seq (o [B,T,H,dv], S_final [B,H,dk,dv], both float64)."""
+    oracle.gdn_seq (o [B,T,H,dv], S_final [B,H,dk,dv], both float64).  With beta_v
+    (FG^2-GDN+, reading notes sec. 2.3 eq. (13)) the values are scaled by sqrt(beta_v)."""
     q = np.asarray(q, dtype=np.float32).astype(np.float64)
     k = np.asarray(k, dtype=np.float32).astype(np.float64)
     v = np.asarray(v, dtype=np.float32).astype(np.float64)
     alpha = np.asarray(alpha, dtype=np.float32).astype(np.float64)
     beta = np.asarray(beta, dtype=np.float32).astype(np.float64)
+    if beta_v is not None:
+        beta_v = np.asarray(beta_v, dtype=np.float32).astype(np.float64)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    if not beta_scalar and dk != dv:
+    if not beta_scalar and beta_v is None and dk != dv:
         raise ValueError("channel-wise beta needs dk == dv")
     o = np.zeros((B, T, H, dv))
     sf = np.zeros((B, H, dk, dv))
@@ -50,12 +53,13 @@ def gdn_chunked(q, k, v, alpha, beta, S0=None, *, chunk, alpha_scalar=False,
             S = np.zeros((dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float32)[b, h].astype(np.float64)
             qh = _normalise(q[b, :, h], eps)
             kh = _normalise(k[b, :, h], eps)
+            src_v = beta if beta_v is None else beta_v
             if beta_scalar:
                 bk = np.repeat(beta[b, :, h][:, None], dk, axis=1)
-                bv = np.repeat(beta[b, :, h][:, None], dv, axis=1)
+                bv = np.repeat(src_v[b, :, h][:, None], dv, axis=1)
             else:
                 bk = beta[b, :, h]
-                bv = beta[b, :, h]
+                bv = src_v[b, :, h]
             al = np.repeat(alpha[b, :, h][:, None], dk, axis=1) if alpha_scalar else alpha[b, :, h]
             kt = np.sqrt(bk) * kh
             vt = np.sqrt(bv) * v[b, :, h]

@@ -32,6 +32,13 @@
  *       channels (reading notes, sec. 1 table of GDN / KDA / FG^2-GDN).
  *     - channel-wise beta multiplies v, so it needs dk == dv (eq. (11)).
  *
+ *   FG^2-GDN+ -- same paper, "FG2-GDN+ Variant"; reading notes sec. 2.3,
+ *   eq. (13): the key side and the value side get their own rates,
+ *       k^_t = sqrt(beta^k_t) (.) k_t,   v~_t = sqrt(beta^v_t) (.) v_t
+ *       S_t  = (I - k^_t k^_t^T) Diag(alpha_t) S_{t-1} + k^_t v~_t^T
+ *   with beta^k in R^{dk} and beta^v in R^{dv} (so dk may differ from dv).
+ *   gdn_head takes an optional beta_v; when it is given, v is scaled by it.
+ *
  *   DeltaProduct -- "DeltaProduct: Improving State-Tracking in Linear RNNs via
  *   Householder Products", "Approach": n_h generalized Householder steps per
  *   token, each one online gradient step on one (k, v, beta) triple,
@@ -66,7 +73,7 @@ static void l2_normalise(const float* x, int n, double eps, double* out) {
 
 /* One (batch, head) pair of the FG^2-GDN recurrence, eq. (11). */
 static void gdn_head(const float* q, const float* k, const float* v,
-                     const float* alpha, const float* beta, const float* S0,
+                     const float* alpha, const float* beta, const float* beta_v, const float* S0,
                      double* o, double* S_final,
                      int b, int h, int B, int H, int T, int dk, int dv,
                      int alpha_scalar, int beta_scalar, double eps) {
@@ -94,7 +101,9 @@ static void gdn_head(const float* q, const float* k, const float* v,
             kt[i] *= sqrt(bi);
         }
         for (int j = 0; j < dv; ++j) {
-            double bj = beta_scalar ? (double)beta[tok] : (double)beta[tok * dk + j];
+            double bj;
+            if (beta_v) bj = beta_scalar ? (double)beta_v[tok] : (double)beta_v[tok * dv + j];
+            else bj = beta_scalar ? (double)beta[tok] : (double)beta[tok * dk + j];
             vt[j] = (double)vr[j] * sqrt(bj);
         }
         /* X = Diag(alpha_t) S_{t-1} */
@@ -129,12 +138,12 @@ static void gdn_head(const float* q, const float* k, const float* v,
 /* Whole tensor, or the (b,h) pairs listed in `pairs` (2*npairs ints) when
  * npairs > 0.  Rows of o / S_final for pairs not listed are left untouched. */
 int oracle_gdn_seq(const float* q, const float* k, const float* v,
-                   const float* alpha, const float* beta, const float* S0,
+                   const float* alpha, const float* beta, const float* beta_v, const float* S0,
                    double* o, double* S_final,
                    int B, int H, int T, int dk, int dv,
                    int alpha_scalar, int beta_scalar, double eps,
                    const int* pairs, int npairs, int nthreads) {
-    if (!beta_scalar && dk != dv) return 1;
+    if (!beta_scalar && !beta_v && dk != dv) return 1;
     int n = npairs > 0 ? npairs : B * H;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -143,7 +152,7 @@ int oracle_gdn_seq(const float* q, const float* k, const float* v,
     for (int p = 0; p < n; ++p) {
         int b = npairs > 0 ? pairs[2 * p] : p / H;
         int h = npairs > 0 ? pairs[2 * p + 1] : p % H;
-        gdn_head(q, k, v, alpha, beta, S0, o, S_final, b, h, B, H, T, dk, dv,
+        gdn_head(q, k, v, alpha, beta, beta_v, S0, o, S_final, b, h, B, H, T, dk, dv,
                  alpha_scalar, beta_scalar, eps);
     }
     return 0;

@@ -452,3 +452,59 @@ def test_deltaproduct_as_interleaved_gdn_sequence():
                                     beta_scalar=True)
         np.testing.assert_allclose(o2[:, nh - 1::nh], o, rtol=0, atol=1e-11)
         np.testing.assert_allclose(s2, s, rtol=0, atol=1e-11)
+
+
+# --------------------------------------------------------------------------- FG^2-GDN+
+def _plus_inputs(seed, T=10, dk=6, dv=9):
+    q, k, v, alpha, beta_k, S0 = _gdn_inputs(seed, T=T, dk=dk, dv=dv)
+    beta_v = _rng(seed + 1000).uniform(0.0, 1.0, (1, T, 2, dv)).astype(np.float32)
+    return q, k, v, alpha, beta_k, beta_v, S0
+
+
+def test_plus_with_equal_rates_is_fg2():
+    """FG^2-GDN+ with beta^v = beta^k is FG^2-GDN (FG^2-GDN summary, "FG2-GDN+ Variant";
+    reading notes sec. 2.3 eq. (13) against eq. (11))."""
+    q, k, v, alpha, beta, S0 = _gdn_inputs(30, T=11)
+    o1, s1 = oracle.gdn_seq(q, k, v, alpha, beta, S0)
+    o2, s2 = oracle.gdn_seq(q, k, v, alpha, beta, S0, beta_v=beta.copy())
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(s1, s2, rtol=0, atol=1e-14)
+
+
+def test_plus_write_identity_and_gradient_step():
+    """Eq. (13): S_t = X + k^ (v~ - X^T k^)^T with k^ = sqrt(beta^k) (.) k and
+    v~ = sqrt(beta^v) (.) v, i.e. one gradient step on 1/2 ||X^T k^ - v~||^2 (autograd);
+    with ||k^|| = 1 the write is exact: S_t^T k^ = v~."""
+    q, k, v, alpha, beta_k, beta_v, S0 = _plus_inputs(31, T=1, dk=5, dv=7)
+    _, S1 = oracle.gdn_seq(q, k, v, alpha, beta_k, S0, beta_v=beta_v, eps=0.0)
+    for h in range(2):
+        kh = torch.tensor(np.sqrt(beta_k[0, 0, h].astype(np.float64)) * _unit(k[0, 0, h]))
+        vt = torch.tensor(np.sqrt(beta_v[0, 0, h].astype(np.float64)) * v[0, 0, h].astype(np.float64))
+        X = torch.tensor(alpha[0, 0, h][:, None].astype(np.float64) * S0[0, h], requires_grad=True)
+        (grad,) = torch.autograd.grad(0.5 * ((X.T @ kh - vt) ** 2).sum(), X)
+        np.testing.assert_allclose(S1[0, h], (X - grad).detach().numpy(), rtol=0, atol=1e-12)
+    ones = np.ones_like(beta_k)
+    _, S1 = oracle.gdn_seq(q, k, v, alpha, ones, S0, beta_v=beta_v, eps=0.0)
+    for h in range(2):
+        vt = np.sqrt(beta_v[0, 0, h].astype(np.float64)) * v[0, 0, h]
+        np.testing.assert_allclose(S1[0, h].T @ _unit(k[0, 0, h]), vt, rtol=0, atol=1e-12)
+
+
+def test_plus_value_rate_scales_linearly():
+    """With S0 = 0 the state and output are linear in v~ = sqrt(beta^v) (.) v, so
+    multiplying beta^v by c^2 multiplies them by c (eq. (13))."""
+    q, k, v, alpha, beta_k, beta_v, _ = _plus_inputs(32, T=12)
+    o1, s1 = oracle.gdn_seq(q, k, v, alpha, beta_k, None, beta_v=beta_v)
+    o2, s2 = oracle.gdn_seq(q, k, v, alpha, beta_k, None, beta_v=4.0 * beta_v)
+    np.testing.assert_allclose(o2, 2.0 * o1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s2, 2.0 * s1, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16])
+def test_plus_sequential_equals_chunked(chunk):
+    """FG^2-GDN+ with dk != dv: token-by-token and chunkwise forms agree."""
+    q, k, v, alpha, beta_k, beta_v, S0 = _plus_inputs(33, T=37, dk=6, dv=9)
+    o1, s1 = oracle.gdn_seq(q, k, v, alpha, beta_k, S0, beta_v=beta_v)
+    o2, s2 = oracle.gdn_chunked(q, k, v, alpha, beta_k, S0, chunk=chunk, beta_v=beta_v)
+    assert np.abs(o1 - o2).max() <= 1e-12 * np.sqrt(np.mean(o1 ** 2))
+    assert np.abs(s1 - s2).max() <= 1e-12 * np.sqrt(np.mean(s1 ** 2))
