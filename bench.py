@@ -181,10 +181,12 @@ def run_reference(args, cfg):
     if rank != 0:
         return
     vals, last = [], None
+    # each step is a bounded sample, sized so that warm-up + timed steps end within minutes
+    budget = max(0.5, min(args.ref_budget, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(max(0, args.warmup)):
-        pass
+        cpu_baseline(cfg, budget_s=budget)
     for _ in range(args.steps):
-        last = cpu_baseline(cfg, budget_s=args.ref_budget)
+        last = cpu_baseline(cfg, budget_s=budget)
         vals.append(last["value"])
     v = float(np.median(vals))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
@@ -210,8 +212,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up + timed steps (no clock soak, e2e or CPU baseline), for ncu")
+    ap.add_argument("--B", type=int, default=None, help="override the workload's batch (small ncu captures)")
+    ap.add_argument("--H", type=int, default=None, help="override the workload's heads")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's tokens per sequence")
     args = ap.parse_args()
     cfg = CONFIGS[args.workload]
+    over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}
+    if over:
+        import dataclasses
+        tag = ",".join(f"{k}={v}" for k, v in over.items())
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}[{tag}]", **over)
     if args.impl == "reference":
         return run_reference(args, cfg)
 

@@ -14,6 +14,15 @@ bool tc_supported(const Problem& p, bool bf16);
 size_t tc_inter_bytes(const Problem& p);
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream);
 int tc_launches(const Problem& p);
+// gdn_decode.cu
+cudaError_t launch_decode(const Problem& p, bool bf16, cudaStream_t stream);
+// gdn_bwd.cu
+bool bwd_supported(int C, int dk, int dv);
+size_t bwd_inter_bytes(const Problem& p, size_t fwd_inter);
+int bwd_launches(const Problem& p);
+cudaError_t launch_bwd(Problem p, const void* dO, const float* dS_final, float* dq, float* dk,
+                       float* dv, float* dalpha, float* dbeta, float* dbeta_v, float* dS0,
+                       size_t fwd_inter, bool bf16, cudaStream_t stream);
 }  // namespace gdn
 
 using namespace gdn;
@@ -28,7 +37,7 @@ bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
 // Fills `p` (without pointers) and checks sizes.  Returns GDN_OK or the error.
 gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int dv, int chunk,
-                          gdn_dtype_t dtype, unsigned flags, bool dp) {
+                          gdn_dtype_t dtype, unsigned flags, bool dp, bool plus = false) {
     if (B < 0 || H < 0 || T < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR)) return GDN_ERR_INVALID_ARG;
@@ -36,7 +45,7 @@ gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int d
     if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
     if (dp && (nh < 1 || nh > 4)) return GDN_ERR_UNSUPPORTED;
     const bool beta_scalar = dp || (flags & GDN_BETA_SCALAR);
-    if (!beta_scalar && dk != dv) return GDN_ERR_INVALID_ARG;
+    if (!beta_scalar && !plus && dk != dv) return GDN_ERR_INVALID_ARG;   // sqrt(beta) scales v too
     if (!simt_supported(chunk, dk, dv)) return GDN_ERR_UNSUPPORTED;
     p = Problem{};
     p.B = B; p.H = H; p.T = T;
@@ -60,7 +69,8 @@ gdn_status_t run(Problem& p, bool bf16, void* workspace, size_t workspace_bytes,
     const bool has_tokens = p.B > 0 && p.H > 0 && p.T > 0;
     if (has_tokens && (!p.q || !p.k || !p.v || !p.alpha || !p.beta || !p.out)) return GDN_ERR_INVALID_ARG;
     if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.alpha) ||
-        !aligned16(p.beta) || !aligned16(p.out) || !aligned16(p.S0) || !aligned16(p.S_final))
+        !aligned16(p.beta) || !aligned16(p.beta_v) || !aligned16(p.out) || !aligned16(p.S0) ||
+        !aligned16(p.S_final))
         return GDN_ERR_INVALID_ARG;
     const size_t need = workspace_bytes_for(p, bf16);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
@@ -118,6 +128,36 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
     return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
 }
 
+int gdn_plus_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                                unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return -1;
+    return launches_for(p, dtype == GDN_BF16);
+}
+
+size_t gdn_plus_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                         gdn_dtype_t dtype, unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return 0;
+    return workspace_bytes_for(p, dtype == GDN_BF16);
+}
+
+gdn_status_t gdn_plus_chunk_fwd(const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta_k, const float* beta_v,
+                                const float* S0, void* out, float* S_final,
+                                int B, int H, int T, int dk, int dv, int chunk,
+                                gdn_dtype_t dtype, unsigned flags,
+                                void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream) {
+    Problem p;
+    gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
+    if (st != GDN_OK) return st;
+    if (B > 0 && H > 0 && T > 0 && !beta_v) return GDN_ERR_INVALID_ARG;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta_k; p.beta_v = beta_v;
+    p.S0 = S0; p.out = out; p.S_final = S_final;
+    return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
+}
+
 size_t gdn_deltaproduct_fwd_workspace_size(int B, int H, int T, int n_h, int dk, int dv,
                                            int chunk, gdn_dtype_t dtype) {
     Problem p;
@@ -138,6 +178,85 @@ gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
     p.q = q; p.k = k; p.v = v; p.alpha = gamma; p.beta = beta;
     p.S0 = S0; p.out = out; p.S_final = S_final;
     return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
+}
+
+size_t gdn_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                    gdn_dtype_t dtype, unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return 0;
+    if (!bwd_supported(chunk, dk, dv)) return 0;
+    return kHeaderBytes + bwd_inter_bytes(p, simt_inter_bytes(p));
+}
+
+int gdn_chunk_bwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                           unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return -1;
+    if (!bwd_supported(chunk, dk, dv)) return -1;
+    return (B == 0 || H == 0) ? 0 : bwd_launches(p);
+}
+
+gdn_status_t gdn_chunk_bwd(const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta_k, const float* beta_v,
+                           const float* S0, const void* dout, const float* dS_final,
+                           float* dq, float* dk_, float* dv_, float* dalpha, float* dbeta_k,
+                           float* dbeta_v, float* dS0,
+                           int B, int H, int T, int dk, int dv, int chunk,
+                           gdn_dtype_t dtype, unsigned flags,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, beta_v != nullptr);
+    if (st != GDN_OK) return st;
+    if (!bwd_supported(chunk, dk, dv)) return GDN_ERR_UNSUPPORTED;
+    if (dbeta_v && !beta_v) return GDN_ERR_INVALID_ARG;
+    const bool has_tokens = B > 0 && H > 0 && T > 0;
+    if (has_tokens && (!q || !k || !v || !alpha || !beta_k || !dout)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, alpha, beta_k, beta_v, S0, dout, dS_final, dq, dk_, dv_,
+                          dalpha, dbeta_k, dbeta_v, dS0};
+    for (const void* x : ptrs)
+        if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
+    const size_t fwd = simt_inter_bytes(p);
+    const size_t need = kHeaderBytes + bwd_inter_bytes(p, fwd);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return GDN_ERR_WORKSPACE;
+    if (B == 0 || H == 0) return GDN_OK;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta_k; p.beta_v = beta_v; p.S0 = S0;
+    p.status = static_cast<int*>(workspace);
+    p.inter = static_cast<char*>(workspace) + kHeaderBytes;
+    cudaError_t e = launch_bwd(p, dout, dS_final, dq, dk_, dv_, dalpha, dbeta_k, dbeta_v, dS0, fwd,
+                               dtype == GDN_BF16, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta_k, const float* beta_v,
+                                const float* S_in, float* S_out, void* out,
+                                int B, int H, int dk, int dv, gdn_dtype_t dtype, unsigned flags,
+                                cudaStream_t stream) {
+    if (B < 0 || H < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR)) return GDN_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
+    const bool beta_scalar = (flags & GDN_BETA_SCALAR) != 0;
+    if (!beta_scalar && !beta_v && dk != dv) return GDN_ERR_INVALID_ARG;
+    if ((size_t)B * H * (dv / 32) > 0x7fffffffull) return GDN_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0) return GDN_OK;
+    if (!q || !k || !v || !alpha || !beta_k || !S_out || !out) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(alpha) || !aligned16(beta_k) ||
+        !aligned16(beta_v) || !aligned16(S_in) || !aligned16(S_out) || !aligned16(out))
+        return GDN_ERR_INVALID_ARG;
+    if (S_in && S_in != S_out) {     // in place is allowed; a partial overlap is not
+        const size_t n = (size_t)B * H * dk * dv;
+        if (S_in < S_out + n && S_out < S_in + n) return GDN_ERR_INVALID_ARG;
+    }
+    Problem p{};
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta_k; p.beta_v = beta_v;
+    p.S0 = S_in; p.S_final = S_out; p.out = out;
+    p.B = B; p.H = H; p.T = 1; p.nh = 1; p.L = 1;
+    p.dk = dk; p.dv = dv; p.C = 1; p.NC = 1;
+    p.alpha_scalar = (flags & GDN_ALPHA_SCALAR) ? 1 : 0;
+    p.beta_scalar = beta_scalar ? 1 : 0;
+    return launch_decode(p, dtype == GDN_BF16, stream) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream) {

@@ -1,0 +1,497 @@
+// gdn_bwd.cu -- chunkwise backward of the FG^2-GDN forward (float32, CUDA cores).
+//
+// Gradients of a loss L(o, S_final) given dO = dL/do and dS_final = dL/dS_final,
+// for the recurrence of eq. (11) of the FG^2-GDN reading notes (sec. 2.2; the
+// split rates of eq. (13), sec. 2.3, when beta_v is given), computed chunkwise as
+// the training half of the chunkwise algorithm (sec. 2.4).
+//
+// Per chunk, with S the state at the chunk start, S' the state at its end and
+// (forward, see gdn_common.cuh)
+//     R = V~ - K_G S,  U = (I + A)^{-1} R,  O = Q_G S + P U,  S' = Diag(e^{g_C}) S + K_E^T U
+// where K_G = K~ (.) e^g, Q_G = Q^ (.) e^g, K_E = K~ (.) e^{g_C - g}, the adjoints are
+//     dU = K_E dS' + P^T dO,   dR = (I + A)^{-T} dU,   dV~ = dR,
+//     dP = lower(dO U^T),      dA = strictly-lower(-dR U^T),
+//     dS = Diag(e^{g_C}) dS' + Q_G^T dO - K_G^T dR  =  M^T dS' + Qe^T dO,
+// with M = Diag(e^{g_C}) - K'^T W the forward's chunk transition and Qe = Q_G - P W.
+// So the state gradient runs backwards over chunks with the forward's own chunk
+// quantities (W, Qe, K', e^{g_C}), column by column like the forward scan, and
+// every chunk's remaining gradients follow in parallel from (S, dS', dO):
+//     dq^_r = e^{g_r} (.) (dO S^T)_r + sum_{i<=r} dP_ri k~_i (.) e^{g_r - g_i}
+//     dk~_r = -e^{g_r} (.) (dR S^T)_r + sum_{i<r} dA_ri k~_i (.) e^{g_r - g_i}        ("+" part)
+//           + sum_{r'>r} dA_r'r k~_r' (.) e^{g_r' - g_r} + sum_{r'>=r} dP_r'r q^_r' (.) e^{g_r' - g_r}
+//           + e^{g_C - g_r} (.) (U dS'^T)_r                                           ("-" part)
+//     dg_r  = q^_r (.) dq^_r + k~_r (.) (dk~+_r - dk~-_r),
+//     dg_C += e^{g_C} (.) rowsum(S (.) dS') + sum_r k~_r (.) e^{g_C - g_r} (.) (U dS'^T)_r
+// and d log alpha_s = sum_{r >= s} dg_r (with dg_C added at the chunk's last row).
+// Last, the chain through v~ = sqrt(beta^v) v, k~ = sqrt(beta^k) k^ and the L2
+// normalisations: dx = (dx^ - x^ (x^ . dx^)) / ||x||.
+//
+// Kernels: the forward's intra role (chunk quantities) and scan role (storing the
+// state at every chunk start), then rev_scan_kernel (dS' at every chunk end, and
+// dS0), then grad_chunk_kernel (one CTA per chunk and head).
+#include "gdn.h"
+#include "gdn_common.cuh"
+
+namespace gdn {
+
+cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream);
+
+namespace bwd {
+
+constexpr int NT = 256;
+constexpr int kNS = 32;          // d_v columns per reverse-scan CTA and per S tile
+constexpr int kLd = kNS + 1;     // padded tile row
+constexpr int kMaxRPT = 16;      // rows per thread in the per-element phase: C * dk / NT
+
+struct Grads {
+    const void* dO;              // [B,T,H,dv], dtype storage
+    const float* dS_final;       // [B,H,dk,dv] or null
+    float* dq;                   // [B,T,H,dk]
+    float* dk;
+    float* dv;                   // [B,T,H,dv]
+    float* dalpha;               // [B,T,H,dk] or [B,T,H]
+    float* dbeta;                // [B,T,H,dk] or [B,T,H]
+    float* dbeta_v;              // [B,T,H,dv] or [B,T,H]; only with beta_v
+    float* dS0;                  // [B,H,dk,dv]
+    float* dS_chunks;            // workspace: dL/dS at every chunk end [B,H,NC,dk,dv]
+};
+
+__host__ __device__ inline size_t rev_smem(int C, int dk) {
+    return sizeof(float) * ((size_t)dk * kNS + (size_t)2 * C * kNS + (size_t)3 * C * dk + dk);
+}
+
+// One CTA per (d_v slice, head); serial over chunks from last to first.
+template <typename Tin>
+__global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
+    const int j0 = blockIdx.x * kNS;
+    const int bh = blockIdx.y;
+    const int b = bh / p.H, h = bh % p.H;
+    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int tid = threadIdx.x;
+    extern __shared__ float sm[];
+    float* dS = sm;                          // dk x kNS
+    float* Y = dS + (size_t)dk * kNS;        // C x kNS: K' dS'
+    float* dOc = Y + (size_t)C * kNS;        // C x kNS
+    float* Wc = dOc + (size_t)C * kNS;       // C x dk
+    float* Qc = Wc + (size_t)C * dk;
+    float* Kc = Qc + (size_t)C * dk;
+    float* gc = Kc + (size_t)C * dk;         // dk
+    const Tin* dO = static_cast<const Tin*>(gr.dO);
+
+    for (int idx = tid; idx < dk * kNS; idx += NT) {
+        const int i = idx / kNS, j = idx % kNS;
+        dS[idx] = gr.dS_final ? gr.dS_final[((size_t)bh * dk + i) * dv + j0 + j] : 0.f;
+    }
+    InterF32 L{C, dk, dv};
+    for (int c = p.NC - 1; c >= 0; --c) {
+        const float* in = static_cast<const float*>(p.inter) + ((size_t)bh * p.NC + c) * L.floats();
+        __syncthreads();
+        float* dst = gr.dS_chunks + ((size_t)bh * p.NC + c) * dk * dv;
+        for (int idx = tid; idx < dk * kNS; idx += NT) {
+            const int i = idx / kNS, j = idx % kNS;
+            dst[(size_t)i * dv + j0 + j] = dS[idx];
+        }
+        for (int idx = tid; idx < C * dk; idx += NT) {
+            Wc[idx] = in[L.W() + idx];
+            Qc[idx] = in[L.Qe() + idx];
+            Kc[idx] = in[L.Kp() + idx];
+        }
+        for (int i = tid; i < dk; i += NT) gc[i] = in[L.gC() + i];
+        for (int idx = tid; idx < C * kNS; idx += NT) {
+            const int r = idx / kNS, j = idx % kNS;
+            const int s = c * C + r;
+            float x = 0.f;
+            if (s < p.L) {
+                const RowRef rr = row_ref(p, b, h, s);
+                if (rr.has_q) x = load_in(dO, rr.tok * dv + j0 + j);
+            }
+            dOc[idx] = x;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * kNS; idx += NT) {
+            const int r = idx / kNS, j = idx % kNS;
+            float acc = 0.f;
+            for (int i = 0; i < dk; ++i) acc += Kc[(size_t)r * dk + i] * dS[(size_t)i * kNS + j];
+            Y[idx] = acc;
+        }
+        __syncthreads();
+        // dS <- Diag(gC) dS' - W^T Y + Qe^T dO   (element (i, j) reads only its own dS')
+        for (int idx = tid; idx < dk * kNS; idx += NT) {
+            const int i = idx / kNS, j = idx % kNS;
+            float acc = gc[i] * dS[idx];
+            for (int r = 0; r < C; ++r)
+                acc += Qc[(size_t)r * dk + i] * dOc[(size_t)r * kNS + j] - Wc[(size_t)r * dk + i] * Y[(size_t)r * kNS + j];
+            dS[idx] = acc;
+        }
+    }
+    __syncthreads();
+    if (gr.dS0) {
+        for (int idx = tid; idx < dk * kNS; idx += NT) {
+            const int i = idx / kNS, j = idx % kNS;
+            gr.dS0[((size_t)bh * dk + i) * dv + j0 + j] = dS[idx];
+        }
+    }
+}
+
+__host__ __device__ inline size_t grad_smem(int C, int dk, int dv) {
+    return sizeof(float) * ((size_t)5 * C * dk + (size_t)4 * C * dv + (size_t)4 * C * C +
+                            (size_t)2 * dk * kLd + 2 * C + dk);
+}
+
+// One CTA per (chunk, head).
+template <typename Tin>
+__global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
+    const int c = blockIdx.x;
+    const int bh = blockIdx.y;
+    const int b = bh / p.H, h = bh % p.H;
+    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int s0 = c * C;
+    const int Cv = min(C, p.L - s0);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int nwarps = NT / 32;
+
+    extern __shared__ float sm[];
+    float* qh = sm;                          // q^                      C x dk
+    float* kt = qh + (size_t)C * dk;         // k~
+    float* g = kt + (size_t)C * dk;          // log alpha, then cumulative
+    float* KG = g + (size_t)C * dk;          // k~ e^g,          later dq^
+    float* KE = KG + (size_t)C * dk;         // k~ e^{g_C - g},  later dk~
+    float* vt = KE + (size_t)C * dk;         // v~                      C x dv
+    float* dOs = vt + (size_t)C * dv;        // dO
+    float* U = dOs + (size_t)C * dv;         // R, then U
+    float* dR = U + (size_t)C * dv;          // K_E dS', then dU, then dR
+    float* A = dR + (size_t)C * dv;          // C x C
+    float* P = A + (size_t)C * C;
+    float* dP = P + (size_t)C * C;
+    float* dA = dP + (size_t)C * C;
+    float* St = dA + (size_t)C * C;          // S tile   dk x kLd,  later dg (C x dk)
+    float* dSt = St + (size_t)dk * kLd;      // dS' tile dk x kLd
+    float* iq = dSt + (size_t)dk * kLd;      // 1 / ||q_r||             C
+    float* ik = iq + C;                      // 1 / ||k_r||             C
+    float* dgC = ik + C;                     // dk
+
+    const Tin* q = static_cast<const Tin*>(p.q);
+    const Tin* k = static_cast<const Tin*>(p.k);
+    const Tin* v = static_cast<const Tin*>(p.v);
+    const Tin* dO = static_cast<const Tin*>(gr.dO);
+    const float* bvsrc = p.beta_v ? p.beta_v : p.beta;
+    const int bvstride = p.beta_v ? dv : dk;
+
+    // 1. rows: q^, k~, v~, log alpha, dO
+    for (int r = warp; r < C; r += nwarps) {
+        float* qr = qh + (size_t)r * dk;
+        float* kr = kt + (size_t)r * dk;
+        float* gq = g + (size_t)r * dk;
+        if (r < Cv) {
+            const RowRef rr = row_ref(p, b, h, s0 + r);
+            float ssq = 0.f, ssk = 0.f;
+            for (int j = lane; j < dk; j += 32) {
+                const float xq = load_in(q, rr.tok * dk + j);
+                const float xk = load_in(k, rr.tok * dk + j);
+                qr[j] = xq;
+                kr[j] = xk;
+                ssq += xq * xq;
+                ssk += xk * xk;
+            }
+            const float a = rsqrtf(warp_sum(ssq) + kNormEps);
+            const float bk = rsqrtf(warp_sum(ssk) + kNormEps);
+            if (lane == 0) {
+                iq[r] = a;
+                ik[r] = bk;
+            }
+            const float bs = p.beta_scalar ? sqrtf(p.beta[rr.tok]) : 0.f;
+            const float la = p.alpha_scalar ? logf(p.alpha[rr.tok]) : 0.f;
+            for (int j = lane; j < dk; j += 32) {
+                qr[j] *= a;
+                kr[j] *= bk * (p.beta_scalar ? bs : sqrtf(p.beta[rr.tok * dk + j]));
+                gq[j] = p.alpha_scalar ? la : logf(p.alpha[rr.tok * dk + j]);
+            }
+            const float bvs = p.beta_scalar ? sqrtf(bvsrc[rr.tok]) : 0.f;
+            for (int j = lane; j < dv; j += 32) {
+                const float sb = p.beta_scalar ? bvs : sqrtf(bvsrc[rr.tok * bvstride + j]);
+                vt[(size_t)r * dv + j] = load_in(v, rr.tok * dv + j) * sb;
+                dOs[(size_t)r * dv + j] = load_in(dO, rr.tok * dv + j);
+            }
+        } else {
+            for (int j = lane; j < dk; j += 32) { qr[j] = 0.f; kr[j] = 0.f; gq[j] = 0.f; }
+            for (int j = lane; j < dv; j += 32) { vt[(size_t)r * dv + j] = 0.f; dOs[(size_t)r * dv + j] = 0.f; }
+            if (lane == 0) { iq[r] = 0.f; ik[r] = 0.f; }
+        }
+    }
+    __syncthreads();
+    for (int j = tid; j < dk; j += NT) {
+        float acc = 0.f;
+        for (int r = 0; r < C; ++r) {
+            acc += g[(size_t)r * dk + j];
+            g[(size_t)r * dk + j] = acc;
+        }
+    }
+    __syncthreads();
+    for (int idx = tid; idx < C * dk; idx += NT) {
+        const int j = idx % dk;
+        const float gl = g[(size_t)(C - 1) * dk + j];
+        KG[idx] = kt[idx] * expf(g[idx]);
+        KE[idx] = kt[idx] * expf(gl - g[idx]);
+    }
+    // 2. A (i < r) and P (i <= r), decay formed element by element
+    for (int pr = warp; pr < C * C; pr += nwarps) {
+        const int r = pr / C, i = pr % C;
+        float a = 0.f, pp = 0.f;
+        if (i <= r) {
+            for (int j = lane; j < dk; j += 32) {
+                const float ke = kt[(size_t)i * dk + j] * expf(g[(size_t)r * dk + j] - g[(size_t)i * dk + j]);
+                pp += qh[(size_t)r * dk + j] * ke;
+                a += kt[(size_t)r * dk + j] * ke;
+            }
+            a = warp_sum(a);
+            pp = warp_sum(pp);
+        }
+        if (lane == 0) {
+            A[pr] = (i < r) ? a : 0.f;
+            P[pr] = pp;
+        }
+    }
+    __syncthreads();
+
+    const float* Sg = p.S_chunks + ((size_t)bh * p.NC + c) * dk * dv;
+    const float* dSg = gr.dS_chunks + ((size_t)bh * p.NC + c) * dk * dv;
+    // 3. R = V~ - K_G S and K_E dS', tile by tile over d_v
+    for (int jt = 0; jt < dv; jt += kNS) {
+        for (int idx = tid; idx < dk * kNS; idx += NT) {
+            const int i = idx / kNS, jj = idx % kNS;
+            St[i * kLd + jj] = Sg[(size_t)i * dv + jt + jj];
+            dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
+        }
+        __syncthreads();
+        for (int idx = tid; idx < C * kNS; idx += NT) {
+            const int r = idx / kNS, jj = idx % kNS;
+            float ks = 0.f, kd = 0.f;
+            for (int i = 0; i < dk; ++i) {
+                ks += KG[(size_t)r * dk + i] * St[i * kLd + jj];
+                kd += KE[(size_t)r * dk + i] * dSt[i * kLd + jj];
+            }
+            U[(size_t)r * dv + jt + jj] = vt[(size_t)r * dv + jt + jj] - ks;
+            dR[(size_t)r * dv + jt + jj] = kd;
+        }
+        __syncthreads();
+    }
+    // 4. U = (I + A)^{-1} R (forward substitution); dU = K_E dS' + P^T dO;
+    //    dR = (I + A)^{-T} dU (back substitution)
+    for (int r = 1; r < C; ++r) {
+        for (int j = tid; j < dv; j += NT) {
+            float acc = U[(size_t)r * dv + j];
+            for (int i = 0; i < r; ++i) acc -= A[(size_t)r * C + i] * U[(size_t)i * dv + j];
+            U[(size_t)r * dv + j] = acc;
+        }
+        __syncthreads();
+    }
+    for (int idx = tid; idx < C * dv; idx += NT) {
+        const int i = idx / dv, j = idx % dv;
+        float acc = dR[idx];
+        for (int r = i; r < C; ++r) acc += P[(size_t)r * C + i] * dOs[(size_t)r * dv + j];
+        dR[idx] = acc;
+    }
+    __syncthreads();
+    for (int r = C - 2; r >= 0; --r) {
+        for (int j = tid; j < dv; j += NT) {
+            float acc = dR[(size_t)r * dv + j];
+            for (int i = r + 1; i < C; ++i) acc -= A[(size_t)i * C + r] * dR[(size_t)i * dv + j];
+            dR[(size_t)r * dv + j] = acc;
+        }
+        __syncthreads();
+    }
+    // 5. dP = lower(dO U^T), dA = strictly-lower(-dR U^T)
+    for (int pr = warp; pr < C * C; pr += nwarps) {
+        const int r = pr / C, i = pr % C;
+        float a = 0.f, pp = 0.f;
+        if (i <= r) {
+            for (int j = lane; j < dv; j += 32) {
+                const float u = U[(size_t)i * dv + j];
+                pp += dOs[(size_t)r * dv + j] * u;
+                a -= dR[(size_t)r * dv + j] * u;
+            }
+            a = warp_sum(a);
+            pp = warp_sum(pp);
+        }
+        if (lane == 0) {
+            dA[pr] = (i < r) ? a : 0.f;
+            dP[pr] = pp;
+        }
+    }
+    // 6. dO S^T, dR S^T, U dS'^T (thread: column cc, rows r0 + rstep * m) and rowsum(S (.) dS')
+    const int cc = tid % dk, r0 = tid / dk, rstep = NT / dk;
+    const int rpt = C * dk / NT;
+    float G1[kMaxRPT], G2[kMaxRPT], G3[kMaxRPT], G4 = 0.f;
+#pragma unroll
+    for (int m = 0; m < kMaxRPT; ++m) { G1[m] = 0.f; G2[m] = 0.f; G3[m] = 0.f; }
+    for (int jt = 0; jt < dv; jt += kNS) {
+        __syncthreads();
+        for (int idx = tid; idx < dk * kNS; idx += NT) {
+            const int i = idx / kNS, jj = idx % kNS;
+            St[i * kLd + jj] = Sg[(size_t)i * dv + jt + jj];
+            dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
+        }
+        __syncthreads();
+        for (int jj = 0; jj < kNS; ++jj) {
+            const float s = St[cc * kLd + jj], ds = dSt[cc * kLd + jj];
+            if (r0 == 0) G4 += s * ds;
+#pragma unroll
+            for (int m = 0; m < kMaxRPT; ++m) {
+                if (m < rpt) {
+                    const size_t o = (size_t)(r0 + rstep * m) * dv + jt + jj;
+                    G1[m] += dOs[o] * s;
+                    G2[m] += dR[o] * s;
+                    G3[m] += U[o] * ds;
+                }
+            }
+        }
+    }
+    __syncthreads();
+    const float gCc = g[(size_t)(C - 1) * dk + cc];
+    if (r0 == 0) dgC[cc] = expf(gCc) * G4;
+    __syncthreads();
+    // 7. dq^, dk~ and dg per element
+    float* Dg = St;
+#pragma unroll
+    for (int m = 0; m < kMaxRPT; ++m) {
+        if (m >= rpt) continue;
+        const int r = r0 + rstep * m;
+        const size_t e = (size_t)r * dk + cc;
+        const float grc = g[e];
+        float dq = expf(grc) * G1[m];
+        float dkp = -expf(grc) * G2[m];
+        float dkm = expf(gCc - grc) * G3[m];
+        const float ke3 = KE[e] * G3[m];
+        for (int i = 0; i <= r; ++i) {
+            const float w = kt[(size_t)i * dk + cc] * expf(grc - g[(size_t)i * dk + cc]);
+            dq += dP[(size_t)r * C + i] * w;
+            if (i < r) dkp += dA[(size_t)r * C + i] * w;
+        }
+        for (int i = r; i < C; ++i) {
+            const float ex = expf(g[(size_t)i * dk + cc] - grc);
+            dkm += dP[(size_t)i * C + r] * qh[(size_t)i * dk + cc] * ex;
+            if (i > r) dkm += dA[(size_t)i * C + r] * kt[(size_t)i * dk + cc] * ex;
+        }
+        atomicAdd(&dgC[cc], ke3);
+        Dg[e] = qh[e] * dq + kt[e] * (dkp - dkm);
+        KG[e] = dq;
+        KE[e] = dkp + dkm;
+    }
+    __syncthreads();
+    // 8. d log alpha = reverse cumulative sum of dg (dg_C at the last row)
+    for (int j = tid; j < dk; j += NT) {
+        float acc = dgC[j];
+        for (int r = C - 1; r >= 0; --r) {
+            acc += Dg[(size_t)r * dk + j];
+            Dg[(size_t)r * dk + j] = acc;
+        }
+    }
+    __syncthreads();
+    // 9. chain through the rates, alpha and the normalisations, one row per warp
+    for (int r = warp; r < Cv; r += nwarps) {
+        const size_t t = row_ref(p, b, h, s0 + r).tok;
+        const float* qr = qh + (size_t)r * dk;
+        const float* dqr = KG + (size_t)r * dk;      // dq^
+        const float* dkr = KE + (size_t)r * dk;      // dk~
+        const float sbk_s = p.beta_scalar ? sqrtf(p.beta[t]) : 0.f;
+        const float sbv_s = p.beta_scalar ? sqrtf(bvsrc[t]) : 0.f;
+        float dotq = 0.f, dotk = 0.f;
+        for (int j = lane; j < dk; j += 32) {
+            const float sb = p.beta_scalar ? sbk_s : sqrtf(p.beta[t * dk + j]);
+            dotq += qr[j] * dqr[j];
+            dotk += load_in(k, t * dk + j) * ik[r] * sb * dkr[j];
+        }
+        dotq = warp_sum(dotq);
+        dotk = warp_sum(dotk);
+        float dbk = 0.f, dbv = 0.f, dal = 0.f;
+        for (int j = lane; j < dk; j += 32) {
+            const float sb = p.beta_scalar ? sbk_s : sqrtf(p.beta[t * dk + j]);
+            const float khat = load_in(k, t * dk + j) * ik[r];
+            if (gr.dq) gr.dq[t * dk + j] = (dqr[j] - qr[j] * dotq) * iq[r];
+            if (gr.dk) gr.dk[t * dk + j] = (sb * dkr[j] - khat * dotk) * ik[r];
+            float db = dkr[j] * khat * 0.5f / sb;             // d sqrt(b) / db = 1 / (2 sqrt(b))
+            if (!p.beta_v && !p.beta_scalar)                   // one rate on k and v (dk == dv)
+                db += dR[(size_t)r * dv + j] * load_in(v, t * dv + j) * 0.5f / sb;
+            if (p.beta_scalar) dbk += db;
+            else if (gr.dbeta) gr.dbeta[t * dk + j] = db;
+            const float dla = Dg[(size_t)r * dk + j];          // d log alpha
+            if (p.alpha_scalar) dal += dla;
+            else if (gr.dalpha) gr.dalpha[t * dk + j] = dla / p.alpha[t * dk + j];
+        }
+        for (int j = lane; j < dv; j += 32) {
+            const float sb = p.beta_scalar ? sbv_s : sqrtf(bvsrc[t * bvstride + j]);
+            const float dvt = dR[(size_t)r * dv + j];
+            if (gr.dv) gr.dv[t * dv + j] = sb * dvt;
+            const float db = dvt * load_in(v, t * dv + j) * 0.5f / sb;
+            if (p.beta_scalar) dbv += db;
+            else if (p.beta_v && gr.dbeta_v) gr.dbeta_v[t * dv + j] = db;
+        }
+        if (p.alpha_scalar) {
+            dal = warp_sum(dal);
+            if (lane == 0 && gr.dalpha) gr.dalpha[t] = dal / p.alpha[t];
+        }
+        if (p.beta_scalar) {
+            dbk = warp_sum(dbk);
+            dbv = warp_sum(dbv);
+            if (lane == 0) {
+                if (p.beta_v) {
+                    if (gr.dbeta) gr.dbeta[t] = dbk;
+                    if (gr.dbeta_v) gr.dbeta_v[t] = dbv;
+                } else if (gr.dbeta) {
+                    gr.dbeta[t] = dbk + dbv;
+                }
+            }
+        }
+    }
+}
+
+template <typename Tin>
+cudaError_t launch_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    const size_t s3 = rev_smem(p.C, p.dk);
+    cudaFuncSetAttribute(rev_scan_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+    rev_scan_kernel<Tin><<<dim3(p.dv / kNS, p.B * p.H), NT, s3, stream>>>(p, gr);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || p.NC == 0) return e;
+    const size_t s4 = grad_smem(p.C, p.dk, p.dv);
+    cudaFuncSetAttribute(grad_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
+    grad_chunk_kernel<Tin><<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
+    return cudaGetLastError();
+}
+
+}  // namespace bwd
+
+bool bwd_supported(int C, int dk, int dv) {
+    return (C == 16 || C == 32) && (size_t)C * dk <= (size_t)bwd::kMaxRPT * bwd::NT &&
+           bwd::grad_smem(C, dk, dv) <= 227 * 1024 && bwd::rev_smem(C, dk) <= 227 * 1024;
+}
+
+// Workspace after the header: the forward's chunk quantities, then the states at
+// every chunk start, then the state gradients at every chunk end (each 256-aligned).
+size_t bwd_inter_bytes(const Problem& p, size_t fwd_inter) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t states = (size_t)p.B * p.H * p.NC * p.dk * p.dv * sizeof(float);
+    return up(fwd_inter) + 2 * up(states);
+}
+
+int bwd_launches(const Problem& p) { return p.NC > 0 ? 4 : 1; }
+
+cudaError_t launch_bwd(Problem p, const void* dO, const float* dS_final, float* dq, float* dk,
+                       float* dv, float* dalpha, float* dbeta, float* dbeta_v, float* dS0,
+                       size_t fwd_inter, bool bf16, cudaStream_t stream) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t states = (size_t)p.B * p.H * p.NC * p.dk * p.dv * sizeof(float);
+    char* base = static_cast<char*>(p.inter);
+    p.S_chunks = reinterpret_cast<float*>(base + up(fwd_inter));
+    bwd::Grads gr{dO, dS_final, dq, dk, dv, dalpha, dbeta, dbeta_v, dS0,
+                  reinterpret_cast<float*>(base + up(fwd_inter) + up(states))};
+    if (p.NC > 0) {
+        Problem f = p;                 // state recompute: no outputs, chunk-start states kept
+        f.out = nullptr;
+        f.S_final = nullptr;
+        cudaError_t e = launch_simt(f, bf16, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return bf16 ? bwd::launch_t<__nv_bfloat16>(p, gr, stream) : bwd::launch_t<float>(p, gr, stream);
+}
+
+}  // namespace gdn

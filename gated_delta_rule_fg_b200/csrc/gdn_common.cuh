@@ -6,7 +6,8 @@
 // Fine-Grained Control", sec. 2.2 eq. (11) and sec. 2.4) is split in two roles:
 //
 //   intra role (independent per chunk): load a chunk of C rows, L2-normalise
-//     q and k, scale k and v by sqrt(beta), take the cumulative log-decay
+//     q and k, scale k and v by sqrt(beta) (FG^2-GDN+, sec. 2.3 eq. (13): k by
+//     sqrt(beta^k) and v by sqrt(beta^v)), take the cumulative log-decay
 //     g_r = sum_{s<=r} log alpha_s per channel, and build
 //       A   = strictly-lower (K~ e^g)(K~ e^-g)^T    P = lower (Q^ e^g)(K~ e^-g)^T
 //       T   = (I + A)^{-1}                          (UT transform)
@@ -37,7 +38,8 @@ struct Problem {
     const void* k;
     const void* v;
     const float* alpha;     // GDN: alpha; DeltaProduct: gamma (scalar per token)
-    const float* beta;
+    const float* beta;      // key rate beta^k (and value rate, unless beta_v is set)
+    const float* beta_v;    // FG^2-GDN+ value rate beta^v (eq. (13)); null: beta scales v too
     const float* S0;        // may be null
     void* out;
     float* S_final;         // may be null
@@ -50,6 +52,8 @@ struct Problem {
     int dp;                 // 1: DeltaProduct row mapping
     int* status;            // workspace header word
     void* inter;            // per-chunk intermediates written by the intra role
+    float* S_chunks;        // backward recompute: state at every chunk start,
+                            // [B,H,NC,dk,dv]; null in the forward
 };
 
 // Row source of sub-step s of head (b, h) (DeltaProduct interleaves n_h

@@ -81,7 +81,9 @@ intra_simt_kernel(Problem p) {
                 gr[j] = as ? ascal : logf(p.alpha[rr.tok * dk + j]);
             }
             for (int j = lane; j < dv; j += 32) {
-                float bj = bs ? bscal : p.beta[rr.tok * dk + j];   // channel-wise beta needs dk == dv
+                float bj;
+                if (p.beta_v) bj = bs ? p.beta_v[rr.tok] : p.beta_v[rr.tok * dv + j];
+                else bj = bs ? bscal : p.beta[rr.tok * dk + j];   // channel-wise beta needs dk == dv
                 vr[j] = load_in(v, krow * dv + j) * sqrtf(bj);
             }
         } else {
@@ -216,6 +218,13 @@ scan_simt_kernel(Problem p) {
     for (int c = 0; c < p.NC; ++c) {
         const float* in = static_cast<const float*>(p.inter) + ((size_t)bh * p.NC + c) * L.floats();
         __syncthreads();   // previous chunk's S update and U reads are done
+        if (p.S_chunks) {
+            float* dst = p.S_chunks + ((size_t)bh * p.NC + c) * dk * dv;
+            for (int idx = tid; idx < dk * NS; idx += kSimtThreads) {
+                const int i = idx / NS, j = idx % NS;
+                dst[(size_t)i * dv + j0 + j] = S[idx];
+            }
+        }
         for (int idx = tid; idx < C * dk; idx += kSimtThreads) {
             Wc[idx] = in[L.W() + idx];
             Qc[idx] = in[L.Qe() + idx];
@@ -234,7 +243,7 @@ scan_simt_kernel(Problem p) {
             }
             U[idx] = in[L.Up() + (size_t)r * dv + j0 + j] - ws;
             const int s = s0 + r;
-            if (s < p.L) {
+            if (out && s < p.L) {     // no outputs in the backward's state recompute
                 RowRef rr = row_ref(p, b, h, s);
                 if (rr.has_q) store_out(out, rr.tok * dv + j0 + j, in[L.PUp() + (size_t)r * dv + j0 + j] + qs);
             }

@@ -110,6 +110,8 @@ __device__ __forceinline__ void record_timeout(int* status) {
 }
 
 // ============================================================================ intra
+// kPlus: FG^2-GDN+ (separate value rate beta^v, eq. (13)).
+template <bool kPlus>
 __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int c = blockIdx.x;
@@ -167,6 +169,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
                 cp_async16(dst + 4, p.beta + rr.tok * D + 8 * o + 4);
             }
             cp_async16(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128), v + krow * D + 8 * o);
+            if (kPlus && !b_scalar) {
+                // beta^v of (r, o) goes to the two R0 slots this thread later overwrites
+                // with its own KG and QG octets (read first, in the same thread)
+                cp_async16(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128), p.beta_v + rr.tok * D + 8 * o);
+                cp_async16(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128), p.beta_v + rr.tok * D + 8 * o + 4);
+            }
         }
     }
     cp_async_commit();
@@ -204,7 +212,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     const float iq = rsqrtf(ssq + kNormEps);
     const float ik = rsqrtf(ssk + kNormEps);
 
-    float la_s = 0.f, b_s = 0.f;
+    float la_s = 0.f, b_s = 0.f, bv_s = 0.f;
     if (valid) {
         if (p.dp) {
             la_s = rr.m == 0 ? __logf(p.alpha[rr.tok]) : 0.f;
@@ -212,6 +220,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         } else {
             if (p.alpha_scalar) la_s = __logf(p.alpha[rr.tok]);
             if (p.beta_scalar) b_s = p.beta[rr.tok];
+            if (kPlus && p.beta_scalar) bv_s = p.beta_v[rr.tok];
         }
     }
     // log alpha, inclusive scan over the 8 rows of this warp (lanes with equal o0)
@@ -270,7 +279,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
-        float g[8], sb[8], fq[8], fk[8], fv[8];
+        float g[8], sb[8], sv[8], fq[8], fk[8], fv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) g[e] = la[j][e] + scr[warp * D + 8 * o + e];
         if (b_scalar || !valid) {
@@ -283,6 +292,19 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             const float4 b1 = *reinterpret_cast<const float4*>(bsrc + 4);
             sb[0] = sqrtf(b0.x); sb[1] = sqrtf(b0.y); sb[2] = sqrtf(b0.z); sb[3] = sqrtf(b0.w);
             sb[4] = sqrtf(b1.x); sb[5] = sqrtf(b1.y); sb[6] = sqrtf(b1.z); sb[7] = sqrtf(b1.w);
+        }
+        if (!kPlus) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sv[e] = sb[e];
+        } else if (b_scalar || !valid) {
+            const float s = valid ? sqrtf(bv_s) : 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sv[e] = s;
+        } else {
+            const float4 b0 = *reinterpret_cast<const float4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
+            const float4 b1 = *reinterpret_cast<const float4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
+            sv[0] = sqrtf(b0.x); sv[1] = sqrtf(b0.y); sv[2] = sqrtf(b0.z); sv[3] = sqrtf(b0.w);
+            sv[4] = sqrtf(b1.x); sv[5] = sqrtf(b1.y); sv[6] = sqrtf(b1.z); sv[7] = sqrtf(b1.w);
         }
         const uint4 vp = valid ? *reinterpret_cast<const uint4*>(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128))
                                : make_uint4(0, 0, 0, 0);
@@ -303,7 +325,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             KG[e] = kt * ex;
             QG[e] = qh * ex;
             KIG[e] = kt * exi;
-            VT[e] = fv[e] * sb[e];
+            VT[e] = fv[e] * sv[e];
             // fallback chunks: e^{-g} may overflow while e^{g_last} underflows, so take the
             // ratio in one exponent there (it is <= 1)
             KP[e] = fallback ? kt * __expf(glast[ch] - g[e]) : kt * exi * fK[ch];
@@ -869,10 +891,11 @@ size_t tc_inter_bytes(const Problem& p) { return (size_t)p.B * p.H * p.NC * tc::
 int tc_launches(const Problem& p) { return p.NC > 0 ? 2 : 1; }
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
-    cudaFuncSetAttribute(tc::intra_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+    auto intra = p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>;
+    cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
     cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
     dim3 g1(p.NC, p.B * p.H);
-    tc::intra_tc_kernel<<<g1, tc::NT, tc::kIntraSmem, stream>>>(p);
+    intra<<<g1, tc::NT, tc::kIntraSmem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g2(tc::J, p.B * p.H);

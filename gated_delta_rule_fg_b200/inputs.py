@@ -12,6 +12,8 @@ S0; DeltaProduct: q, k, v, beta, gamma-logits):
   alpha    = exp(-s * softplus(x)), x ~ N(0, 1), s = 0.1 (0.02 for near-1 decay)
   beta     = sigmoid(x), x ~ N(0, std)      (std 1, or 2 for the wide config)
   S0       = 0, or ~ N(0, std 0.01)
+  beta_v   = sigmoid(x), x ~ N(0, std)      (FG^2-GDN+ only; drawn last, after S0,
+                                             [B,T,H,dv], or [B,T,H] with scalar beta)
   DeltaProduct: beta ~ U[0, 2] per sub-step, gamma = sigmoid(x), x ~ N(2, 1)
 bf16 tensors are rounded to nearest-even from the float32 draws; the float32
 copy kept alongside holds exactly the rounded values.
@@ -64,6 +66,7 @@ class GdnConfig:
     beta_scalar: bool = False
     s0_std: float = 0.0              # 0 -> S0 is None
     deltaproduct_nh: int = 0         # > 0 -> DeltaProduct with this many sub-steps
+    plus: bool = False               # FG^2-GDN+: a separate value rate beta_v
     seed: int = 0
     extra: dict = field(default_factory=dict)
 
@@ -124,4 +127,8 @@ def make_inputs(cfg: GdnConfig, *, seed: int | None = None, T: int | None = None
     S0 = None
     if cfg.s0_std > 0:
         S0 = (cfg.s0_std * rng.standard_normal((B, H, cfg.dk, cfg.dv), dtype=f32)).astype(f32)
-    return dict(q=q, k=k, v=v, alpha=alpha, beta=beta, S0=S0)
+    x = dict(q=q, k=k, v=v, alpha=alpha, beta=beta, S0=S0)
+    if cfg.plus:
+        vshape = (B, T, H) if cfg.beta_scalar else (B, T, H, cfg.dv)
+        x["beta_v"] = _sigmoid(cfg.beta_std * rng.standard_normal(vshape, dtype=f32)).astype(f32)
+    return x

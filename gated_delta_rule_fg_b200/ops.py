@@ -30,11 +30,20 @@ SIGNATURES = {
                            ctypes.c_uint, _P, _SZ, _P]),
     "gdn_chunk_fwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                    ctypes.c_uint, _P]),
+    "gdn_plus_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
+    "gdn_plus_chunk_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                ctypes.c_uint, _P, _SZ, _P]),
+    "gdn_plus_chunk_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_deltaproduct_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_deltaproduct_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                   _I, _P, _SZ, _P]),
     "gdn_chunk_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_deltaproduct_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "gdn_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                ctypes.c_uint, _P]),
+    "gdn_chunk_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
+    "gdn_chunk_bwd": (_I, [_P] * 16 + [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint, _P, _SZ, _P]),
+    "gdn_chunk_bwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_workspace_status": (_I, [_P, _P]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_version": (_I, []),
@@ -101,6 +110,14 @@ def chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
     return int(lib().gdn_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags))
 
 
+def plus_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
+    return int(lib().gdn_plus_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags))
+
+
+def plus_chunk_fwd_launches(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
+    return int(lib().gdn_plus_chunk_fwd_launches(B, H, T, dk, dv, chunk, dtype_code, flags))
+
+
 def deltaproduct_fwd_workspace_size(B, H, T, nh, dk, dv, chunk, dtype_code) -> int:
     return int(lib().gdn_deltaproduct_fwd_workspace_size(B, H, T, nh, dk, dv, chunk, dtype_code))
 
@@ -148,6 +165,37 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=False, be
                              _ptr(workspace), workspace.numel(), _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
+    return out, S_final
+
+
+def plus_chunk_fwd(q, k, v, alpha, beta_k, beta_v, S0=None, *, chunk=64, alpha_scalar=False,
+                   beta_scalar=False, out=None, S_final=None, want_state=True, workspace=None,
+                   stream=None):
+    """FG^2-GDN+ chunkwise forward through gdn_plus_chunk_fwd: beta_k scales the keys
+    and beta_v ([B,T,H,dv], or [B,T,H] with beta_scalar) the values.  Otherwise as
+    chunk_fwd."""
+    code = _dtype_code(q)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype)
+    for t, n in ((alpha, "alpha"), (beta_k, "beta_k"), (beta_v, "beta_v"), (S0, "S0")):
+        _check(t, n, torch.float32)
+    flags = (GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype)
+    _check(S_final, "S_final", torch.float32)
+    need = plus_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, code, flags)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().gdn_plus_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v),
+                                  _ptr(S0), _ptr(out), _ptr(S_final), B, H, T, dk, dv, chunk, code,
+                                  flags, _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_plus_chunk_fwd")
     return out, S_final
 
 
@@ -202,6 +250,85 @@ def deltaproduct_fwd(q, k, v, gamma, beta, S0=None, *, chunk=64, out=None, S_fin
     if st != GDN_OK:
         raise GdnError(st, "gdn_deltaproduct_fwd")
     return out, S_final
+
+
+def chunk_bwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
+    return int(lib().gdn_chunk_bwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags))
+
+
+def chunk_bwd_launches(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
+    return int(lib().gdn_chunk_bwd_launches(B, H, T, dk, dv, chunk, dtype_code, flags))
+
+
+def chunk_bwd(q, k, v, alpha, beta, S0, dout, dS_final=None, *, beta_v=None, chunk=32,
+              alpha_scalar=False, beta_scalar=False, workspace=None, stream=None):
+    """Backward of chunk_fwd / plus_chunk_fwd through gdn_chunk_bwd.
+
+    Same inputs as the forward plus the cotangents dout ([B,T,H,dv], q's dtype) and
+    dS_final (float32 [B,H,dk,dv] or None).  Returns a dict of float32 gradients:
+    q, k, v, alpha, beta (and beta_v when given), S0.
+    """
+    code = _dtype_code(q)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _check(t, n, q.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta"), (beta_v, "beta_v"), (S0, "S0"),
+                 (dS_final, "dS_final")):
+        _check(t, n, torch.float32)
+    flags = (GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"q": torch.empty((B, T, H, dk), **f32), "k": torch.empty((B, T, H, dk), **f32),
+         "v": torch.empty((B, T, H, dv), **f32), "alpha": torch.empty(alpha.shape, **f32),
+         "beta": torch.empty(beta.shape, **f32), "S0": torch.empty((B, H, dk, dv), **f32)}
+    if beta_v is not None:
+        g["beta_v"] = torch.empty(beta_v.shape, **f32)
+    need = chunk_bwd_workspace_size(B, H, T, dk, dv, chunk, code, flags)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().gdn_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(beta_v), _ptr(S0),
+                             _ptr(dout), _ptr(dS_final), _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]),
+                             _ptr(g["alpha"]), _ptr(g["beta"]), _ptr(g.get("beta_v")), _ptr(g["S0"]),
+                             B, H, T, dk, dv, chunk, code, flags, _ptr(workspace), workspace.numel(),
+                             _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_bwd")
+    return g
+
+
+def recurrent_step(q, k, v, alpha, beta_k, S_in=None, *, beta_v=None, alpha_scalar=False,
+                   beta_scalar=False, out=None, S_out=None, in_place=False, stream=None):
+    """One recurrent (decode) step through gdn_recurrent_step.
+
+    q, k [B,H,dk], v [B,H,dv] (bf16 or float32); alpha/beta_k float32 [B,H,dk] or [B,H];
+    beta_v float32 [B,H,dv] / [B,H] or None; S_in float32 [B,H,dk,dv] or None.  With
+    in_place=True the new state overwrites S_in.  Returns (out [B,H,dv], S_out).
+    """
+    code = _dtype_code(q)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype)
+    for t, n in ((alpha, "alpha"), (beta_k, "beta_k"), (beta_v, "beta_v"), (S_in, "S_in")):
+        _check(t, n, torch.float32)
+    flags = (GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    if S_out is None:
+        if in_place:
+            if S_in is None:
+                raise ValueError("in_place needs S_in")
+            S_out = S_in
+        else:
+            S_out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype)
+    _check(S_out, "S_out", torch.float32)
+    st = lib().gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta_k), _ptr(beta_v),
+                                  _ptr(S_in), _ptr(S_out), _ptr(out), B, H, dk, dv, code, flags,
+                                  _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_recurrent_step")
+    return out, S_out
 
 
 def workspace_status(workspace, stream=None) -> int:

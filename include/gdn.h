@@ -125,6 +125,31 @@ gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                    gdn_dtype_t dtype, unsigned flags,
                                    cudaStream_t stream);
 
+/* Bytes of workspace gdn_plus_chunk_fwd needs (0 if invalid/unsupported). */
+size_t gdn_plus_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                         gdn_dtype_t dtype, unsigned flags);
+
+/* FG^2-GDN+ chunkwise forward (same paper, "FG2-GDN+ Variant"; reading notes
+ * sec. 2.3, eq. (13)).  The write rate is split into a key rate beta^k and a
+ * value rate beta^v:
+ *     k~_t = sqrt(beta^k_t) (.) k^_t,   v~_t = sqrt(beta^v_t) (.) v_t
+ *     S_t  = (I - k~_t k~_t^T) Diag(alpha_t) S_{t-1} + k~_t v~_t^T,   o_t = S_t^T q^_t
+ * so the erase acts along beta^k-scaled key directions and the write carries
+ * beta^v-scaled values.
+ *   beta_k: float32 [B,T,H,dk] ([B,T,H] with GDN_BETA_SCALAR), in [0,1].
+ *   beta_v: float32 [B,T,H,dv] ([B,T,H] with GDN_BETA_SCALAR), in [0,1];
+ *           GDN_BETA_SCALAR applies to both rates.
+ * Everything else (layouts, flags, sizes, workspace, paths, errors) is as for
+ * gdn_chunk_fwd, except that channel-wise rates allow dk != dv.  With
+ * beta_v == beta_k the result is gdn_chunk_fwd's. */
+gdn_status_t gdn_plus_chunk_fwd(const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta_k, const float* beta_v,
+                                const float* S0, void* out, float* S_final,
+                                int B, int H, int T, int dk, int dv, int chunk,
+                                gdn_dtype_t dtype, unsigned flags,
+                                void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
 /* Bytes of workspace gdn_deltaproduct_fwd needs (0 if invalid/unsupported). */
 size_t gdn_deltaproduct_fwd_workspace_size(int B, int H, int T, int n_h, int dk, int dv,
                                            int chunk, gdn_dtype_t dtype);
@@ -150,12 +175,71 @@ gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
                                   void* workspace, size_t workspace_bytes,
                                   cudaStream_t stream);
 
-/* Number of kernels one gdn_chunk_fwd / gdn_deltaproduct_fwd call with these
- * sizes enqueues (-1 if the sizes are invalid or unsupported). */
+/* Number of kernels one gdn_chunk_fwd / gdn_plus_chunk_fwd / gdn_deltaproduct_fwd
+ * call with these sizes enqueues (-1 if the sizes are invalid or unsupported). */
 int gdn_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
                            unsigned flags);
+int gdn_plus_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                                unsigned flags);
 int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
                                   gdn_dtype_t dtype);
+
+/* Bytes of workspace gdn_chunk_bwd needs (0 if invalid/unsupported). */
+size_t gdn_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                    gdn_dtype_t dtype, unsigned flags);
+
+/* Chunkwise backward of gdn_chunk_fwd / gdn_plus_chunk_fwd (the training half of
+ * the chunkwise algorithm, reading notes sec. 2.4; the forward is eq. (11), or
+ * eq. (13) when beta_v != NULL).  Given the forward's inputs and the cotangents
+ * dout = dL/dout and dS_final = dL/dS_final, it writes the gradients of L:
+ *   dq, dk [B,T,H,dk]; dv [B,T,H,dv]; dalpha and dbeta_k shaped like alpha and
+ *   beta_k; dbeta_v shaped like beta_v; dS0 [B,H,dk,dv].  All float32.
+ * With beta_v == NULL, dbeta_k is the gradient of the single rate beta (it gets
+ * both the key and the value parts) and dbeta_v must be NULL.  Any gradient
+ * pointer may be NULL (not written); dS_final == NULL means zero; S0 == NULL
+ * means a zero initial state (dS0 is still its gradient).
+ *   q, k, v, dout: dtype storage; alpha, beta_k, beta_v, S0, dS_final: float32.
+ * The forward is recomputed inside (its chunk quantities and the state at every
+ * chunk start are kept in the workspace), in float32 on CUDA cores for both
+ * dtypes.  Sizes: as gdn_chunk_fwd, with chunk in {16, 32} (the backward's own
+ * chunk; the result does not depend on it beyond rounding).  beta in (0, 1]:
+ * the derivative of sqrt(beta) is unbounded at beta = 0.  No device-side waits.
+ * Errors as gdn_chunk_fwd. */
+gdn_status_t gdn_chunk_bwd(const void* q, const void* k, const void* v,
+                           const float* alpha, const float* beta_k, const float* beta_v,
+                           const float* S0, const void* dout, const float* dS_final,
+                           float* dq, float* dk, float* dv, float* dalpha, float* dbeta_k,
+                           float* dbeta_v, float* dS0,
+                           int B, int H, int T, int dk_dim, int dv_dim, int chunk,
+                           gdn_dtype_t dtype, unsigned flags,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of kernels one gdn_chunk_bwd call enqueues (-1 if invalid/unsupported). */
+int gdn_chunk_bwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                           unsigned flags);
+
+/* One recurrent step (single-token decode) for every (b, h): eq. (11) of the
+ * reading notes (sec. 2.2) for one token, with the split rates of eq. (13)
+ * when beta_v is given:
+ *     S_out = (I - k~ k~^T) Diag(alpha) S_in + k~ v~^T,   out = S_out^T q^
+ * with q^, k^, k~, v~ as above (v~ = sqrt(beta_v) (.) v, or sqrt(beta_k) (.) v
+ * when beta_v == NULL).  This continues a sequence whose state came from
+ * gdn_chunk_fwd / gdn_plus_chunk_fwd (their S_final) or from earlier steps.
+ *   q, k [B,H,dk]; v, out [B,H,dv]: dtype storage (one token, no T axis).
+ *   alpha, beta_k: float32 [B,H,dk] ([B,H] with GDN_ALPHA_SCALAR /
+ *   GDN_BETA_SCALAR); beta_v: float32 [B,H,dv] ([B,H] with GDN_BETA_SCALAR) or
+ *   NULL (then channel-wise beta_k needs dk == dv).
+ *   S_in: float32 [B,H,dk,dv] or NULL (zero state); S_out: float32 [B,H,dk,dv].
+ *   S_out may equal S_in (update in place); other overlaps are invalid.
+ * Sizes: B, H >= 0 (0 is a no-op); dk, dv in {32, 64, 128}.  Arithmetic is
+ * float32 for both dtypes.  No workspace: one kernel, no device-side waits.
+ * Errors: GDN_ERR_INVALID_ARG / GDN_ERR_UNSUPPORTED before anything is
+ * enqueued, GDN_ERR_CUDA if the launch fails. */
+gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
+                                const float* alpha, const float* beta_k, const float* beta_v,
+                                const float* S_in, float* S_out, void* out,
+                                int B, int H, int dk, int dv, gdn_dtype_t dtype, unsigned flags,
+                                cudaStream_t stream);
 
 /* Waits for `stream`, then returns (and clears) the first device-side error
  * recorded in `workspace` by earlier calls: GDN_OK, GDN_ERR_TIMEOUT or

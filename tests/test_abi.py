@@ -102,3 +102,67 @@ def test_deltaproduct_validation(L):
 
 def test_status_query_needs_workspace(L):
     assert L.gdn_workspace_status(None, None) == ops.GDN_ERR_WORKSPACE
+
+
+def test_plus_validation(L):
+    """gdn_plus_chunk_fwd: channel-wise rates allow dk != dv; beta_v is required and
+    checked for alignment; errors come back before anything is enqueued."""
+    pws = ops.plus_chunk_fwd_workspace_size
+    assert pws(1, 2, 100, 64, 128, 32, ops.GDN_F32, 0) > 0       # dk != dv with channel-wise rates
+    assert ops.chunk_fwd_workspace_size(1, 2, 100, 64, 128, 32, ops.GDN_F32, 0) == 0
+    assert pws(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == \
+        ops.chunk_fwd_workspace_size(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0)
+    assert ops.plus_chunk_fwd_launches(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == 2
+    assert pws(1, 1, 10, 96, 96, 64, ops.GDN_F32, 0) == 0
+
+    def call(beta_v=FAKE, **kw):
+        a = dict(B=1, H=1, T=8, dk=64, dv=64, chunk=64, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.gdn_plus_chunk_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, beta_v, None, FAKE, None,
+                                    a["B"], a["H"], a["T"], a["dk"], a["dv"], a["chunk"],
+                                    ops.GDN_F32, 0, a["ws"], a["wsb"], None)
+
+    assert call(beta_v=None) == ops.GDN_ERR_INVALID_ARG
+    assert call(beta_v=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG
+    assert call(dk=96, dv=96) == ops.GDN_ERR_UNSUPPORTED
+    assert call(ws=None) == ops.GDN_ERR_WORKSPACE
+    assert call(B=0) == ops.GDN_OK
+
+
+def test_recurrent_step_validation(L):
+    f = L.gdn_recurrent_step
+
+    def call(q=FAKE, beta_v=None, S_in=None, S_out=FAKE, out=FAKE, B=1, H=1, dk=64, dv=64, flags=0,
+             dtype=ops.GDN_F32):
+        return f(q, FAKE, FAKE, FAKE, FAKE, beta_v, S_in, S_out, out, B, H, dk, dv, dtype, flags, None)
+
+    assert call(q=None) == ops.GDN_ERR_INVALID_ARG
+    assert call(S_out=None) == ops.GDN_ERR_INVALID_ARG
+    assert call(out=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG
+    assert call(dk=64, dv=128) == ops.GDN_ERR_INVALID_ARG              # channel-wise beta on v
+    assert call(dk=96, dv=96) == ops.GDN_ERR_UNSUPPORTED
+    assert call(dtype=5) == ops.GDN_ERR_INVALID_ARG
+    assert call(flags=4) == ops.GDN_ERR_INVALID_ARG
+    assert call(S_in=FAKE + 256, S_out=FAKE) == ops.GDN_ERR_INVALID_ARG  # partial overlap
+    assert call(B=-1) == ops.GDN_ERR_INVALID_ARG
+    assert call(B=0) == ops.GDN_OK
+
+
+def test_backward_validation(L):
+    bws = ops.chunk_bwd_workspace_size
+    assert bws(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) > 0
+    assert bws(1, 2, 100, 64, 64, 64, ops.GDN_F32, 0) == 0          # chunk 64 not in the backward
+    assert bws(1, 2, 100, 128, 128, 16, ops.GDN_BF16, 0) > 0
+    assert ops.chunk_bwd_launches(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) == 4
+    assert ops.chunk_bwd_launches(1, 2, 0, 64, 64, 32, ops.GDN_F32, 0) == 1
+
+    def call(dbeta_v=None, beta_v=None, dout=FAKE, chunk=32, ws=FAKE):
+        return L.gdn_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, beta_v, None, dout, None, FAKE, FAKE,
+                               FAKE, FAKE, FAKE, dbeta_v, FAKE, 1, 1, 8, 64, 64, chunk, ops.GDN_F32, 0,
+                               ws, 1 << 30, None)
+
+    assert call(dout=None) == ops.GDN_ERR_INVALID_ARG
+    assert call(dbeta_v=FAKE) == ops.GDN_ERR_INVALID_ARG              # dbeta_v without beta_v
+    assert call(chunk=64) == ops.GDN_ERR_UNSUPPORTED
+    assert call(ws=None) == ops.GDN_ERR_WORKSPACE
+    assert call(dout=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG

@@ -178,3 +178,58 @@ def test_tensor_core_strong_decay_fallback():
     x = make_inputs(cfg)
     x["alpha"] = np.where(np.arange(200)[None, :, None, None] % 3 == 0, 1e-6, x["alpha"]).astype(np.float32)
     check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+# --------------------------------------------------------------------------- FG^2-GDN+
+def run_plus(cfg, x, chunk=None):
+    ops = _ops()
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    out, sf = ops.plus_chunk_fwd(to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt),
+                                 to_dev(x["alpha"]), to_dev(x["beta"]), to_dev(x["beta_v"]),
+                                 to_dev(x["S0"]), chunk=chunk or cfg.chunk,
+                                 alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), sf.cpu().numpy()
+
+
+def oracle_plus(cfg, x, pairs=None):
+    return oracle.gdn_seq(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], beta_v=x["beta_v"],
+                          alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar, pairs=pairs)
+
+
+PLUS = [("f32", 64, 64, 16, 131), ("f32", 32, 64, 32, 70), ("f32", 128, 32, 64, 100),
+        ("bf16", 64, 64, 32, 250), ("bf16", 128, 128, 64, 1), ("bf16", 128, 128, 64, 63),
+        ("bf16", 128, 128, 64, 65), ("bf16", 128, 128, 64, 200)]
+
+
+@pytest.mark.parametrize("dtype,dk,dv,chunk,T", PLUS)
+@pytest.mark.parametrize("scalar", [False, True])
+def test_plus_small(dtype, dk, dv, chunk, T, scalar):
+    """FG^2-GDN+ (separate beta^k / beta^v): CUDA-core and tensor-core shapes, dk != dv,
+    ragged tails, scalar and channel-wise rates; nonzero S0 on odd T."""
+    cfg = GdnConfig("plus", B=2, H=2, T=T, dk=dk, dv=dv, chunk=chunk, dtype=dtype, plus=True,
+                    beta_scalar=scalar, s0_std=0.1 if T % 2 else 0.0, seed=3000 + T + dk)
+    x = make_inputs(cfg)
+    check(cfg, run_plus(cfg, x), oracle_plus(cfg, x))
+
+
+def test_plus_equal_rates_matches_fg2_call():
+    """gdn_plus_chunk_fwd with beta_v = beta_k returns gdn_chunk_fwd's result bit for bit."""
+    cfg = GdnConfig("plus_eq", B=1, H=4, T=300, dk=128, dv=128, chunk=64, plus=True, s0_std=0.05,
+                    seed=3100)
+    x = make_inputs(cfg)
+    x["beta_v"] = x["beta"].copy()
+    o1, s1 = run_plus(cfg, x)
+    o2, s2 = run_gdn(cfg, x)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+def test_plus_full_size_sampled_heads():
+    """FG^2-GDN+ on the 32K-token prefill shape; sampled heads against the oracle."""
+    base = CONFIGS["fg2_prefill_32k"]
+    cfg = GdnConfig("plus_prefill_32k", B=base.B, H=base.H, T=base.T, dk=base.dk, dv=base.dv,
+                    chunk=base.chunk, plus=True, seed=3200)
+    x = make_inputs(cfg)
+    pairs = [(0, 0), (0, cfg.H - 1)]
+    check(cfg, run_plus(cfg, x), oracle_plus(cfg, x, pairs=pairs), pairs=pairs)
