@@ -83,11 +83,16 @@ def load_traffic(kernel: str, workload: str, source_hash: str):
     return float(e["dram_bytes_per_launch"])
 
 
+TC_SOURCES = ("gdn_tc.cu", "gdn_sm100.cuh")     # the timed kernels' own code
+
+
 def source_hash() -> str:
+    """Hash of the sources of the kernels bench.py times; traffic counters taken on other
+    sources are not reported."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_fg_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
+    for n in TC_SOURCES:
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode())
             h.update(f.read())

@@ -54,6 +54,8 @@ struct Problem {
     void* inter;            // per-chunk intermediates written by the intra role
     float* S_chunks;        // backward recompute: state at every chunk start,
                             // [B,H,NC,dk,dv]; null in the forward
+    int prefetch_ahead;     // intra role: CTAs per wave (SMs x resident CTAs); each CTA warms
+                            // L2 with the inputs of the CTA this far ahead in launch order
 };
 
 // Row source of sub-step s of head (b, h) (DeltaProduct interleaves n_h

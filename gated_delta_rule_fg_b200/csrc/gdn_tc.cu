@@ -276,6 +276,32 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     __half* fb_k = reinterpret_cast<__half*>(blk + kOffPU);               // k~ fp16 [C][D]
     __half* fb_q = reinterpret_cast<__half*>(blk + kOffN);                // q^ fp16 [C][D]
     cp_async_wait_all();     // this thread's own staged beta and v
+    // The CTAs of one wave load together and then compute with HBM idle.  Now that this
+    // CTA's inputs have arrived, start the next wave's: the CTA prefetch_ahead places
+    // later in launch order (x = chunk fastest) finds its rows in L2.
+    {
+        const long nxt = (long)blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
+        if (p.prefetch_ahead > 0 && nxt < (long)gridDim.x * gridDim.y) {
+            const int c2 = (int)(nxt % gridDim.x), bh2 = (int)(nxt / gridDim.x);
+            const int r2 = tid >> 2, part = tid & 3;        // 4 threads per row
+            const int s2 = c2 * C + r2;
+            if (s2 < p.L) {
+                const RowRef rp = row_ref(p, bh2 / p.H, bh2 % p.H, s2);
+                const size_t kr2 = p.dp ? rp.tok * p.nh + rp.m : rp.tok;
+                // 128-byte lines: q, k, v rows 2 each (bf16), alpha / beta / beta_v rows 4 each
+                if (part < 2) {
+                    if (rp.has_q) prefetch_l2(q + rp.tok * D + 64 * part);
+                    prefetch_l2(k + kr2 * D + 64 * part);
+                    prefetch_l2(v + kr2 * D + 64 * part);
+                }
+                if (!a_scalar) prefetch_l2(p.alpha + rp.tok * D + 32 * part);
+                if (!b_scalar) {
+                    prefetch_l2(p.beta + rp.tok * D + 32 * part);
+                    if (kPlus) prefetch_l2(p.beta_v + rp.tok * D + 32 * part);
+                }
+            }
+        }
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
@@ -893,9 +919,19 @@ int tc_launches(const Problem& p) { return p.NC > 0 ? 2 : 1; }
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>;
     cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+    Problem pi = p;
+    {
+        int dev = 0, sms = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra, tc::NT, tc::kIntraSmem) == cudaSuccess)
+            pi.prefetch_ahead = sms * per_sm;
+        else
+            pi.prefetch_ahead = 0;
+    }
     cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
     dim3 g1(p.NC, p.B * p.H);
-    intra<<<g1, tc::NT, tc::kIntraSmem, stream>>>(p);
+    intra<<<g1, tc::NT, tc::kIntraSmem, stream>>>(pi);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     dim3 g2(tc::J, p.B * p.H);
