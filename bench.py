@@ -205,6 +205,127 @@ def run_reference(args, cfg):
     print(json.dumps(line))
 
 
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest of every rank's x (each rank passes its own): all-reduce MAX."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(units_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank (weak scaling)."""
+    return units_per_rank * world / (ms_per_step / 1000.0)
+
+
+class Op:
+    """What one bench step runs: device inputs, the step, and the numbers that describe it."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def _fwd_bytes(cfg, plus=False):
+    return algorithmic_bytes(cfg) + (cfg.B * cfg.T * cfg.H * (4 if cfg.beta_scalar else 4 * cfg.dv)
+                                      if plus else 0)
+
+
+def build_op(args, cfg, ops, torch, dev, stream, rank):
+    """Inputs (resident in HBM, one replica per rank with its own seed) and the step for --op."""
+    import dataclasses
+    from gated_delta_rule_fg_b200.inputs import GdnConfig, round_bf16
+    op = args.op
+    if op == "plus":
+        cfg = dataclasses.replace(cfg, plus=True, name=cfg.name + "+plus")
+    if op == "decode":
+        B = args.B if args.B is not None else 256
+        H = args.H if args.H is not None else cfg.H
+        cfg = GdnConfig(f"decode_b{B}_h{H}_d{cfg.dk}", B=B, H=H, T=1, dk=cfg.dk, dv=cfg.dv, chunk=cfg.chunk,
+                        dtype=cfg.dtype, s0_std=0.01, seed=6)
+    x = make_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    if op == "decode":      # one token: drop the T axis
+        x = {k: (np.ascontiguousarray(v[:, 0]) if (v is not None and k != "S0") else v) for k, v in x.items()}
+    if op == "bwd":
+        r = np.random.default_rng(cfg.seed + 7)
+        dO = r.standard_normal((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=np.float32)
+        x["dO"] = round_bf16(dO) if cfg.dtype == "bf16" else dO
+    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+    host = {k: (torch.from_numpy(v).pin_memory() if v is not None else None) for k, v in x.items()}
+    for kname in ("q", "k", "v", "dO"):
+        if kname in host:
+            host[kname] = host[kname].to(dt).pin_memory()
+    d = {k: (v.to(dev, non_blocking=False) if v is not None else None) for k, v in host.items()}
+    dp = cfg.deltaproduct_nh > 0
+    code = ops.GDN_BF16 if cfg.dtype == "bf16" else ops.GDN_F32
+    B, T, H = cfg.B, cfg.T, cfg.H
+    flags = (ops.GDN_ALPHA_SCALAR if cfg.alpha_scalar else 0) | (ops.GDN_BETA_SCALAR if cfg.beta_scalar else 0)
+    e = 2 if cfg.dtype == "bf16" else 4
+    th = B * T * H
+
+    if op == "decode":
+        S = d["S0"]
+        o = torch.empty((B, H, cfg.dv), dtype=dt, device=dev)
+
+        def step(src):
+            ops.recurrent_step(src["q"], src["k"], src["v"], src["alpha"], src["beta"], S, in_place=True,
+                               out=o, stream=stream)
+        per_head = 2 * cfg.dk * cfg.dv * 4 + (2 * cfg.dk + 2 * cfg.dv) * e + 2 * cfg.dk * 4
+        return Op(cfg=cfg, d=d, host=host, step=step, launches=1, ws=None,
+                  abytes=B * H * per_head, flops=float(B * H * 6 * cfg.dk * cfg.dv), tokens=B,
+                  metric=f"tokens/s FG²-GDN decode step (B={B} sequences, H={H}, d={cfg.dk}), 1 B200",
+                  e2e_in=["q", "k", "v", "alpha", "beta"], e2e_out=[o], kernel="gdn_recurrent_step")
+    if op == "bwd":
+        chunk = 16
+        nws = ops.chunk_bwd_workspace_size(B, H, T, cfg.dk, cfg.dv, chunk, code, flags)
+        ws = ops.alloc_workspace(nws, dev)
+        res = {}
+
+        def step(src):
+            res["g"] = ops.chunk_bwd(src["q"], src["k"], src["v"], src["alpha"], src["beta"], src["S0"], src["dO"],
+                                     None, chunk=chunk, alpha_scalar=cfg.alpha_scalar,
+                                     beta_scalar=cfg.beta_scalar, workspace=ws, stream=stream)
+        per = (2 * cfg.dk + cfg.dv) * e + cfg.dv * e + 2 * cfg.dk * 4 + (3 * cfg.dk + cfg.dv) * 4 + 4 * cfg.dk
+        return Op(cfg=cfg, d=d, host=host, step=step, ws=ws,
+                  launches=ops.chunk_bwd_launches(B, H, T, cfg.dk, cfg.dv, chunk, code, flags),
+                  abytes=th * per + B * H * cfg.dk * cfg.dv * 4 * (2 if cfg.s0_std > 0 else 1),
+                  flops=3.0 * algorithmic_flops(cfg), tokens=B * T,
+                  metric=f"tokens/s FG²-GDN chunked bwd (T={T}, d={cfg.dk}, chunk {chunk}), 1 B200",
+                  e2e_in=None, e2e_out=None, kernel="gdn_chunk_bwd")
+
+    out = torch.empty((B, T, H, cfg.dv), dtype=dt, device=dev)
+    Sf = torch.empty((B, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+    if dp:
+        nws = ops.deltaproduct_fwd_workspace_size(B, H, T, cfg.deltaproduct_nh, cfg.dk, cfg.dv, cfg.chunk, code)
+        launches = ops.deltaproduct_fwd_launches(B, H, T, cfg.deltaproduct_nh, cfg.dk, cfg.dv, cfg.chunk, code)
+    elif op == "plus":
+        nws = ops.plus_chunk_fwd_workspace_size(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
+        launches = ops.plus_chunk_fwd_launches(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
+    else:
+        nws = ops.chunk_fwd_workspace_size(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
+        launches = ops.chunk_fwd_launches(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
+    ws = ops.alloc_workspace(nws, dev)
+
+    def step(src):
+        if dp:
+            ops.deltaproduct_fwd(src["q"], src["k"], src["v"], src["gamma"], src["beta"], src["S0"],
+                                 chunk=cfg.chunk, out=out, S_final=Sf, workspace=ws, stream=stream)
+        elif op == "plus":
+            ops.plus_chunk_fwd(src["q"], src["k"], src["v"], src["alpha"], src["beta"], src["beta_v"], src["S0"],
+                               chunk=cfg.chunk, alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar,
+                               out=out, S_final=Sf, workspace=ws, stream=stream)
+        else:
+            ops.chunk_fwd(src["q"], src["k"], src["v"], src["alpha"], src["beta"], src["S0"],
+                          chunk=cfg.chunk, alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar,
+                          out=out, S_final=Sf, workspace=ws, stream=stream)
+    names = ["q", "k", "v", "gamma" if dp else "alpha", "beta"] + (["beta_v"] if op == "plus" else []) + ["S0"]
+    metric = METRIC if op == "fwd" else "tokens/s FG²-GDN+ chunked fwd (T=32K, d=128) and % of roofline, 1 B200"
+    return Op(cfg=cfg, d=d, host=host, step=step, ws=ws, launches=launches,
+              abytes=_fwd_bytes(cfg, op == "plus"), flops=algorithmic_flops(cfg), tokens=B * T,
+              metric=metric, e2e_in=names, e2e_out=[out, Sf], kernel="gdn_chunk_fwd")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -212,6 +333,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="fg2_prefill_32k", choices=sorted(CONFIGS))
+    ap.add_argument("--op", default="fwd", choices=["fwd", "plus", "decode", "bwd"],
+                    help="fwd: the chunked forward (the headline); plus: FG²-GDN+ forward; decode: one "
+                         "recurrent step per sequence (B=256 by default); bwd: the chunked backward")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -223,7 +347,7 @@ def main():
     args = ap.parse_args()
     cfg = CONFIGS[args.workload]
     over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}
-    if over:
+    if over and args.op != "decode":
         import dataclasses
         tag = ",".join(f"{k}={v}" for k, v in over.items())
         cfg = dataclasses.replace(cfg, name=f"{cfg.name}[{tag}]", **over)
@@ -244,35 +368,8 @@ def main():
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
 
-    # ---- inputs (resident in HBM), one replica per rank with its own seed
-    x = make_inputs(cfg, seed=cfg.seed + 1000 * rank)
-    dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-    host = {k: (torch.from_numpy(v).pin_memory() if v is not None else None) for k, v in x.items()}
-    for kname in ("q", "k", "v"):
-        host[kname] = host[kname].to(dt).pin_memory()
-    d = {k: (v.to(dev, non_blocking=False) if v is not None else None) for k, v in host.items()}
-    dp = cfg.deltaproduct_nh > 0
-    code = ops.GDN_BF16 if cfg.dtype == "bf16" else ops.GDN_F32
-    B, T, H = cfg.B, cfg.T, cfg.H
-    out = torch.empty((B, T, H, cfg.dv), dtype=dt, device=dev)
-    Sf = torch.empty((B, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
-    if dp:
-        nws = ops.deltaproduct_fwd_workspace_size(B, H, T, cfg.deltaproduct_nh, cfg.dk, cfg.dv, cfg.chunk, code)
-        launches = ops.deltaproduct_fwd_launches(B, H, T, cfg.deltaproduct_nh, cfg.dk, cfg.dv, cfg.chunk, code)
-    else:
-        flags = (ops.GDN_ALPHA_SCALAR if cfg.alpha_scalar else 0) | (ops.GDN_BETA_SCALAR if cfg.beta_scalar else 0)
-        nws = ops.chunk_fwd_workspace_size(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
-        launches = ops.chunk_fwd_launches(B, H, T, cfg.dk, cfg.dv, cfg.chunk, code, flags)
-    ws = ops.alloc_workspace(nws, dev)
-
-    def step(src):
-        if dp:
-            ops.deltaproduct_fwd(src["q"], src["k"], src["v"], src["gamma"], src["beta"], src["S0"],
-                                 chunk=cfg.chunk, out=out, S_final=Sf, workspace=ws, stream=stream)
-        else:
-            ops.chunk_fwd(src["q"], src["k"], src["v"], src["alpha"], src["beta"], src["S0"],
-                          chunk=cfg.chunk, alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar,
-                          out=out, S_final=Sf, workspace=ws, stream=stream)
+    op = build_op(args, cfg, ops, torch, dev, stream, rank)
+    cfg, d, host, step, ws = op.cfg, op.d, op.host, op.step, op.ws
 
     def barrier():
         if world > 1:
@@ -281,7 +378,8 @@ def main():
 
     for _ in range(max(3, args.warmup)):
         step(d)
-    assert ops.workspace_status(ws) == ops.GDN_OK
+    if ws is not None:
+        assert ops.workspace_status(ws) == ops.GDN_OK
 
     # ---- device-resident timed region (inputs >> L2, so every step streams from HBM)
     clocks = ClockSampler(local)
@@ -306,66 +404,65 @@ def main():
     clk = clocks.stop() if not args.profile else None
     total_ms = e0.elapsed_time(e1)
     per_call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    status = ops.workspace_status(ws)
-    if status != ops.GDN_OK:
-        raise SystemExit(f"device status after the timed region: {ops.status_string(status)}")
-    t_max = torch.tensor([total_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    if ws is not None:
+        status = ops.workspace_status(ws)
+        if status != ops.GDN_OK:
+            raise SystemExit(f"device status after the timed region: {ops.status_string(status)}")
+    total_ms = max_over_ranks(total_ms, dev, world)
     ms_per_step = total_ms / args.steps
-    tokens = B * T * world
-    value = tokens / (ms_per_step / 1000.0)
+    tokens = op.tokens * world
+    value = whole_job_value(op.tokens, world, ms_per_step)
 
     # ---- end to end through the C ABI with pinned host buffers
-    names = ["q", "k", "v", "gamma" if dp else "alpha", "beta", "S0"]
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names if host[n] is not None)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    sf_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
-    d2h = out_h.numel() * out_h.element_size() + sf_h.numel() * sf_h.element_size()
-    dev_in = {n: (torch.empty_like(d[n]) if d[n] is not None else None) for n in names}
-    barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(0 if args.profile else args.e2e_steps):
+    e2e = None
+    if op.e2e_in is not None:
+        names = op.e2e_in
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names if host[n] is not None)
+        outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in op.e2e_out]
+        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+        dev_in = dict(d)
         for n in names:
-            if host[n] is not None:
-                dev_in[n].copy_(host[n], non_blocking=True)
-        step(dev_in)
-        out_h.copy_(out, non_blocking=True)
-        sf_h.copy_(Sf, non_blocking=True)
-    f1.record(stream)
-    barrier()
-    e2e_ms = f0.elapsed_time(f1) / max(1, args.e2e_steps)
-    t_e = torch.tensor([e2e_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t_e, op=dist.ReduceOp.MAX)
-    e2e_value = tokens / (float(t_e.item()) / 1000.0)
+            dev_in[n] = torch.empty_like(d[n]) if d[n] is not None else None
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(0 if args.profile else args.e2e_steps):
+            for n in names:
+                if host[n] is not None:
+                    dev_in[n].copy_(host[n], non_blocking=True)
+            step(dev_in)
+            for th_, td_ in zip(outs_h, op.e2e_out):
+                th_.copy_(td_, non_blocking=True)
+        f1.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / max(1, args.e2e_steps), dev, world)
+        e2e = {"value": whole_job_value(op.tokens, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
 
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
-    abytes = algorithmic_bytes(cfg)
+    abytes = op.abytes
     achieved = abytes / (per_call_ms / 1000.0) / 1e9
-    kname = "gdn_chunk_fwd" if launches == 1 else f"gdn_chunk_fwd ({launches} kernels, whole call)"
+    kname = op.kernel if op.launches == 1 else f"{op.kernel} ({op.launches} kernels, whole call)"
+    traffic = load_traffic(op.kernel, cfg.name, source_hash()) if args.op == "fwd" else None
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
-            "frac": achieved / hbm_gbs, "traffic": load_traffic("gdn_chunk_fwd", cfg.name, source_hash()),
+            "frac": achieved / hbm_gbs, "traffic": traffic,
             "peak_kind": f"of {peak_kind} copy bandwidth", "kernel": kname,
-            "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": algorithmic_flops(cfg),
-            "flop_frac_of_bf16_peak": algorithmic_flops(cfg) / (per_call_ms / 1000.0) / (bf16_tf * 1e12),
+            "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": op.flops,
+            "flop_frac_of_bf16_peak": op.flops / (per_call_ms / 1000.0) / (bf16_tf * 1e12),
             "launch_ms": per_call_ms}
 
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    line = {"metric": op.metric, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded numpy draws with the workload's distributions)",
-            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
+            "config": {"workload": cfg.name, "op": args.op, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
                        "dv": cfg.dv, "chunk": cfg.chunk, "per_rank": "one replica per GPU",
                        "l2": f"inputs larger than L2 ({abytes / 1e9:.2f} GB per step vs {L2_BYTES / 2**20:.0f} MiB)"},
             "roofline": roof,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                    "d2h_bytes_per_step": int(d2h)},
-            "gpu_launches": int(launches * args.steps),
+            "e2e": e2e if e2e is not None else {"value": None, "unit": "tokens/s", "note": "measured for the forward ops only"},
+            "gpu_launches": int(op.launches * args.steps),
             "clocks": clk}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
+    if rank == 0 and world == 1 and args.op == "fwd" and not args.no_cpu_baseline and not args.profile:
         cb = cpu_baseline(cfg)
         cb.pop("seconds", None)
         line["cpu_baseline"] = cb
