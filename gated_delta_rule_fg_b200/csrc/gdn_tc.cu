@@ -159,6 +159,23 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     // into a staging area over R3..R6 (free until the solve), v straight into its final
     // place in R2 (converted in place later).  Everything is issued before any arithmetic.
     float* bstage = reinterpret_cast<float*>(sm + kR3);
+    // Without beta^v, raw q and k also go to shared memory, into the R0 slots this thread
+    // later overwrites with its own QG and KG octets; they are the first commit group, so
+    // the norms wait for them alone.  (Holding them in registers through the norm and
+    // prefix phases costs 32 registers and forces spills.)
+    if (!kPlus) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int o = o0 + 4 * j;
+            uint8_t* kdst = sm + kR0 + off_kmajor(r, 8 * o, 2048, 128);
+            uint8_t* qdst = sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128);
+            if (valid) cp_async16(kdst, k + krow * D + 8 * o);
+            else *reinterpret_cast<uint4*>(kdst) = make_uint4(0, 0, 0, 0);
+            if (valid && rr.has_q) cp_async16(qdst, q + rr.tok * D + 8 * o);
+            else *reinterpret_cast<uint4*>(qdst) = make_uint4(0, 0, 0, 0);
+        }
+        cp_async_commit();
+    }
     if (valid) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -183,8 +200,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
-        qp[j] = (valid && rr.has_q) ? ldg16(q + rr.tok * D + 8 * o) : make_uint4(0, 0, 0, 0);
-        kp[j] = valid ? ldg16(k + krow * D + 8 * o) : make_uint4(0, 0, 0, 0);
+        if (kPlus) {
+            qp[j] = (valid && rr.has_q) ? ldg16(q + rr.tok * D + 8 * o) : make_uint4(0, 0, 0, 0);
+            kp[j] = valid ? ldg16(k + krow * D + 8 * o) : make_uint4(0, 0, 0, 0);
+        }
         if (valid && !a_scalar) {
             al0[j] = ldg16f(p.alpha + rr.tok * D + 8 * o);
             al1[j] = ldg16f(p.alpha + rr.tok * D + 8 * o + 4);
@@ -193,10 +212,16 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             al1[j] = al0[j];
         }
     }
+    if (!kPlus) cp_async_wait_group<1>();      // q and k (the older group) have landed
     float ssq = 0.f, ssk = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
+        const int o = o0 + 4 * j;
         float fq[8], fk[8];
+        if (!kPlus) {
+            qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
+            kp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
+        }
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
 #pragma unroll
@@ -334,6 +359,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         }
         const uint4 vp = valid ? *reinterpret_cast<const uint4*>(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128))
                                : make_uint4(0, 0, 0, 0);
+        if (!kPlus) {      // reread from shared memory: not held in registers across the phases
+            qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
+            kp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
+        }
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
         bf8_to_f(vp, fv);
