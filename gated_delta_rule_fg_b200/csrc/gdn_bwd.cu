@@ -42,6 +42,9 @@ constexpr int NT = 256;
 constexpr int kNS = 32;          // d_v columns per reverse-scan CTA and per S tile
 constexpr int kLd = kNS + 1;     // padded tile row
 constexpr int kMaxRPT = 16;      // rows per thread in the per-element phase: C * dk / NT
+constexpr int kGroups = NT / kNS;              // 8 threads per column in the reverse scan
+// Kernels are instantiated per rows-per-thread (NR = C / 8, NI = dk / 8 in the reverse
+// scan; RPT = C * dk / 256 in the gradient kernel) so unrolled loops have no idle steps.
 
 struct Grads {
     const void* dO;              // [B,T,H,dv], dtype storage
@@ -60,70 +63,126 @@ __host__ __device__ inline size_t rev_smem(int C, int dk) {
     return sizeof(float) * ((size_t)dk * kNS + (size_t)2 * C * kNS + (size_t)3 * C * dk + dk);
 }
 
-// One CTA per (d_v slice, head); serial over chunks from last to first.
-template <typename Tin>
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(dst)),
+                 "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_floats(float* dst, const float* src, int n, int tid) {
+    for (int i = 4 * tid; i < n; i += 4 * NT) cp16(dst + i, src + i);
+}
+__device__ __forceinline__ void commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void wait_all_but_newest() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// One CTA per (d_v slice, head); serial over chunks from last to first.  Per chunk:
+// Y = K' dS' (phase A), then dS = Diag(e^{g_C}) dS' - W^T Y + Qe^T dO (phase B).  The
+// chunk quantities are fetched one phase ahead with asynchronous copies: K' of chunk c-1
+// while phase B of c runs, and W, Qe, e^{g_C}, dO of c-1 while phase A of c-1 runs.
+template <typename Tin, int NR, int NI>
 __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
     const int j0 = blockIdx.x * kNS;
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int tid = threadIdx.x;
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* dS = sm;                          // dk x kNS
     float* Y = dS + (size_t)dk * kNS;        // C x kNS: K' dS'
-    float* dOc = Y + (size_t)C * kNS;        // C x kNS
+    float* dOc = Y + (size_t)C * kNS;        // C x kNS slots: raw dO rows (Tin)
     float* Wc = dOc + (size_t)C * kNS;       // C x dk
     float* Qc = Wc + (size_t)C * dk;
     float* Kc = Qc + (size_t)C * dk;
     float* gc = Kc + (size_t)C * dk;         // dk
     const Tin* dO = static_cast<const Tin*>(gr.dO);
+    Tin* dOs = reinterpret_cast<Tin*>(dOc);
+    constexpr int kRowChunks = kNS * (int)sizeof(Tin) / 16;   // 16-byte pieces of one row slice
+
+    InterF32 L{C, dk, dv};
+    const float* inter = static_cast<const float*>(p.inter);
+    auto block = [&](int c) { return inter + ((size_t)bh * p.NC + c) * L.floats(); };
+    auto fetch_a = [&](int c) {
+        if (c >= 0) cp_floats(Kc, block(c) + L.Kp(), C * dk, tid);
+        commit_group();
+    };
+    auto fetch_b = [&](int c) {
+        if (c >= 0) {
+            const float* in = block(c);
+            cp_floats(Wc, in + L.W(), C * dk, tid);
+            cp_floats(Qc, in + L.Qe(), C * dk, tid);
+            cp_floats(gc, in + L.gC(), dk, tid);
+            for (int i = tid; i < C * kRowChunks; i += NT) {
+                const int r = i / kRowChunks, q16 = i % kRowChunks;
+                const int s = c * C + r;
+                Tin* dst = dOs + (size_t)r * kNS;
+                bool ok = false;
+                if (s < p.L) {
+                    const RowRef rr = row_ref(p, b, h, s);
+                    if (rr.has_q) {
+                        cp16(reinterpret_cast<char*>(dst) + 16 * q16,
+                             reinterpret_cast<const char*>(dO + rr.tok * dv + j0) + 16 * q16);
+                        ok = true;
+                    }
+                }
+                if (!ok) *reinterpret_cast<uint4*>(reinterpret_cast<char*>(dst) + 16 * q16) = make_uint4(0, 0, 0, 0);
+            }
+        }
+        commit_group();
+    };
 
     for (int idx = tid; idx < dk * kNS; idx += NT) {
         const int i = idx / kNS, j = idx % kNS;
         dS[idx] = gr.dS_final ? gr.dS_final[((size_t)bh * dk + i) * dv + j0 + j] : 0.f;
     }
-    InterF32 L{C, dk, dv};
+    fetch_a(p.NC - 1);
+    fetch_b(p.NC - 1);
     for (int c = p.NC - 1; c >= 0; --c) {
-        const float* in = static_cast<const float*>(p.inter) + ((size_t)bh * p.NC + c) * L.floats();
-        __syncthreads();
+        wait_all_but_newest();               // K' of chunk c
+        __syncthreads();                     // ... for all; dS' of chunk c is complete
         float* dst = gr.dS_chunks + ((size_t)bh * p.NC + c) * dk * dv;
         for (int idx = tid; idx < dk * kNS; idx += NT) {
             const int i = idx / kNS, j = idx % kNS;
             dst[(size_t)i * dv + j0 + j] = dS[idx];
         }
-        for (int idx = tid; idx < C * dk; idx += NT) {
-            Wc[idx] = in[L.W() + idx];
-            Qc[idx] = in[L.Qe() + idx];
-            Kc[idx] = in[L.Kp() + idx];
-        }
-        for (int i = tid; i < dk; i += NT) gc[i] = in[L.gC() + i];
-        for (int idx = tid; idx < C * kNS; idx += NT) {
-            const int r = idx / kNS, j = idx % kNS;
-            const int s = c * C + r;
-            float x = 0.f;
-            if (s < p.L) {
-                const RowRef rr = row_ref(p, b, h, s);
-                if (rr.has_q) x = load_in(dO, rr.tok * dv + j0 + j);
+        {   // thread: column j, rows rg, rg + 8, ...; each dS'[i][j] read once for all its rows
+            const int j = tid % kNS, rg = tid / kNS;
+            float acc[NR];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) acc[m] = 0.f;
+            for (int i = 0; i < dk; ++i) {
+                const float x = dS[(size_t)i * kNS + j];
+#pragma unroll
+                for (int m = 0; m < NR; ++m) acc[m] += Kc[(size_t)(rg + kGroups * m) * dk + i] * x;
             }
-            dOc[idx] = x;
+#pragma unroll
+            for (int m = 0; m < NR; ++m) Y[(size_t)(rg + kGroups * m) * kNS + j] = acc[m];
         }
-        __syncthreads();
-        for (int idx = tid; idx < C * kNS; idx += NT) {
-            const int r = idx / kNS, j = idx % kNS;
-            float acc = 0.f;
-            for (int i = 0; i < dk; ++i) acc += Kc[(size_t)r * dk + i] * dS[(size_t)i * kNS + j];
-            Y[idx] = acc;
-        }
+        __syncthreads();                     // K' buffer free; Y complete
+        fetch_a(c - 1);
+        wait_all_but_newest();               // W, Qe, e^{g_C}, dO of chunk c
         __syncthreads();
         // dS <- Diag(gC) dS' - W^T Y + Qe^T dO   (element (i, j) reads only its own dS')
-        for (int idx = tid; idx < dk * kNS; idx += NT) {
-            const int i = idx / kNS, j = idx % kNS;
-            float acc = gc[i] * dS[idx];
-            for (int r = 0; r < C; ++r)
-                acc += Qc[(size_t)r * dk + i] * dOc[(size_t)r * kNS + j] - Wc[(size_t)r * dk + i] * Y[(size_t)r * kNS + j];
-            dS[idx] = acc;
+        {   // thread: column j, state rows ig, ig + 8, ...; dO[r][j], Y[r][j] read once
+            const int j = tid % kNS, ig = tid / kNS;
+            float acc[NI];
+#pragma unroll
+            for (int m = 0; m < NI; ++m) {
+                const int i = ig + kGroups * m;
+                acc[m] = gc[i] * dS[(size_t)i * kNS + j];
+            }
+            for (int r = 0; r < C; ++r) {
+                const float d = load_in(dOs, (size_t)r * kNS + j), y = Y[(size_t)r * kNS + j];
+#pragma unroll
+                for (int m = 0; m < NI; ++m) {
+                    const int i = ig + kGroups * m;
+                    acc[m] += Qc[(size_t)r * dk + i] * d - Wc[(size_t)r * dk + i] * y;
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < NI; ++m) dS[(size_t)(ig + kGroups * m) * kNS + j] = acc[m];
         }
+        __syncthreads();                     // W, Qe, e^{g_C}, dO buffers free
+        fetch_b(c - 1);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (gr.dS0) {
         for (int idx = tid; idx < dk * kNS; idx += NT) {
@@ -139,7 +198,7 @@ __host__ __device__ inline size_t grad_smem(int C, int dk, int dv) {
 }
 
 // One CTA per (chunk, head).
-template <typename Tin>
+template <typename Tin, int RPT>
 __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
@@ -320,10 +379,9 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     }
     // 6. dO S^T, dR S^T, U dS'^T (thread: column cc, rows r0 + rstep * m) and rowsum(S (.) dS')
     const int cc = tid % dk, r0 = tid / dk, rstep = NT / dk;
-    const int rpt = C * dk / NT;
-    float G1[kMaxRPT], G2[kMaxRPT], G3[kMaxRPT], G4 = 0.f;
+    float G1[RPT], G2[RPT], G3[RPT], G4 = 0.f;
 #pragma unroll
-    for (int m = 0; m < kMaxRPT; ++m) { G1[m] = 0.f; G2[m] = 0.f; G3[m] = 0.f; }
+    for (int m = 0; m < RPT; ++m) { G1[m] = 0.f; G2[m] = 0.f; G3[m] = 0.f; }
     for (int jt = 0; jt < dv; jt += kNS) {
         __syncthreads();
         for (int idx = tid; idx < dk * kNS; idx += NT) {
@@ -336,13 +394,11 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
             const float s = St[cc * kLd + jj], ds = dSt[cc * kLd + jj];
             if (r0 == 0) G4 += s * ds;
 #pragma unroll
-            for (int m = 0; m < kMaxRPT; ++m) {
-                if (m < rpt) {
-                    const size_t o = (size_t)(r0 + rstep * m) * dv + jt + jj;
-                    G1[m] += dOs[o] * s;
-                    G2[m] += dR[o] * s;
-                    G3[m] += U[o] * ds;
-                }
+            for (int m = 0; m < RPT; ++m) {
+                const size_t o = (size_t)(r0 + rstep * m) * dv + jt + jj;
+                G1[m] += dOs[o] * s;
+                G2[m] += dR[o] * s;
+                G3[m] += U[o] * ds;
             }
         }
     }
@@ -353,8 +409,7 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     // 7. dq^, dk~ and dg per element
     float* Dg = St;
 #pragma unroll
-    for (int m = 0; m < kMaxRPT; ++m) {
-        if (m >= rpt) continue;
+    for (int m = 0; m < RPT; ++m) {
         const int r = r0 + rstep * m;
         const size_t e = (size_t)r * dk + cc;
         const float grc = g[e];
@@ -445,17 +500,44 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     }
 }
 
+template <typename Tin, int NR, int NI>
+cudaError_t launch_rev(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    const size_t s3 = rev_smem(p.C, p.dk);
+    cudaFuncSetAttribute(rev_scan_kernel<Tin, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+    rev_scan_kernel<Tin, NR, NI><<<dim3(p.dv / kNS, p.B * p.H), NT, s3, stream>>>(p, gr);
+    return cudaGetLastError();
+}
+
+template <typename Tin, int NR>
+cudaError_t launch_rev_nr(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    switch (p.dk / kGroups) {
+        case 4: return launch_rev<Tin, NR, 4>(p, gr, stream);
+        case 8: return launch_rev<Tin, NR, 8>(p, gr, stream);
+        case 16: return launch_rev<Tin, NR, 16>(p, gr, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename Tin, int RPT>
+cudaError_t launch_grad(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    const size_t s4 = grad_smem(p.C, p.dk, p.dv);
+    cudaFuncSetAttribute(grad_chunk_kernel<Tin, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
+    grad_chunk_kernel<Tin, RPT><<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
+    return cudaGetLastError();
+}
+
 template <typename Tin>
 cudaError_t launch_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
-    const size_t s3 = rev_smem(p.C, p.dk);
-    cudaFuncSetAttribute(rev_scan_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
-    rev_scan_kernel<Tin><<<dim3(p.dv / kNS, p.B * p.H), NT, s3, stream>>>(p, gr);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = (p.C / kGroups == 2) ? launch_rev_nr<Tin, 2>(p, gr, stream)
+                  : (p.C / kGroups == 4) ? launch_rev_nr<Tin, 4>(p, gr, stream) : cudaErrorInvalidValue;
     if (e != cudaSuccess || p.NC == 0) return e;
-    const size_t s4 = grad_smem(p.C, p.dk, p.dv);
-    cudaFuncSetAttribute(grad_chunk_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
-    grad_chunk_kernel<Tin><<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
-    return cudaGetLastError();
+    switch (p.C * p.dk / NT) {
+        case 2: return launch_grad<Tin, 2>(p, gr, stream);
+        case 4: return launch_grad<Tin, 4>(p, gr, stream);
+        case 8: return launch_grad<Tin, 8>(p, gr, stream);
+        case 16: return launch_grad<Tin, 16>(p, gr, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace bwd

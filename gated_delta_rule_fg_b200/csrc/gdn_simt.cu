@@ -9,6 +9,9 @@ namespace gdn {
 
 constexpr int kSimtThreads = 256;
 constexpr int kScanCols = 32;   // d_v columns of the state owned by one scan CTA
+constexpr int kRowGroups = kSimtThreads / kScanCols;   // 8: threads per column in the scan
+// The scan kernel is instantiated per (chunk rows, state rows) a thread carries:
+// NR = C / 8 and NI = dk / 8, so its unrolled loops carry no idle iterations.
 
 // Shared memory of the intra kernel: qh, kt, g (C x dk), vt, Up (C x dv), A, Tm, P (C x C).
 __host__ __device__ inline size_t intra_simt_smem(int C, int dk, int dv) {
@@ -186,12 +189,38 @@ intra_simt_kernel(Problem p) {
     }
 }
 
+// Shared memory of the scan kernel: S (dk x NS), U and the U', PU' slices (C x NS each),
+// W, Qe, K' (C x dk each), e^{g_C} (dk).
 __host__ __device__ inline size_t scan_simt_smem(int C, int dk) {
-    return sizeof(float) * ((size_t)dk * kScanCols + (size_t)C * kScanCols + (size_t)3 * C * dk + dk);
+    return sizeof(float) * ((size_t)dk * kScanCols + (size_t)3 * C * kScanCols + (size_t)3 * C * dk + dk);
 }
 
-// One CTA per (d_v slice of kScanCols columns, head); serial over chunks.
-template <typename Tout>
+// 16-byte asynchronous copy of n floats (n % 4 == 0, both sides 16-byte aligned), spread
+// over the CTA's threads.
+__device__ __forceinline__ void cp_async_floats(float* dst, const float* src, int n, int tid) {
+    for (int i = 4 * tid; i < n; i += 4 * kSimtThreads)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(dst + i)),
+                     "l"(src + i) : "memory");
+}
+// Rows of a column slice: rows x 32 floats from a row-major source of row stride ld.
+__device__ __forceinline__ void cp_async_slice(float* dst, const float* src, int rows, int ld, int tid) {
+    for (int i = tid; i < rows * (kScanCols / 4); i += kSimtThreads) {
+        const int r = i / (kScanCols / 4), q4 = i % (kScanCols / 4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                     ::"r"((unsigned)__cvta_generic_to_shared(dst + r * kScanCols + 4 * q4)),
+                     "l"(src + (size_t)r * ld + 4 * q4) : "memory");
+    }
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// One CTA per (d_v slice of kScanCols columns, head); serial over chunks.  The chunk
+// quantities are fetched one phase ahead with asynchronous copies: W, Qe, U', PU' (used
+// only by the U / output phase) for chunk c+1 while the state update of chunk c runs, and
+// K', e^{g_C} (used only by the state update) for chunk c+1 while the U phase of c+1 runs.
+// Every iteration commits both groups (possibly empty), so "all but the newest group have
+// landed" always names the one needed next.
+template <typename Tout, int NR, int NI>
 __global__ void __launch_bounds__(kSimtThreads)
 scan_simt_kernel(Problem p) {
     const int j0 = blockIdx.x * kScanCols;
@@ -201,23 +230,48 @@ scan_simt_kernel(Problem p) {
     const int tid = threadIdx.x;
     constexpr int NS = kScanCols;
 
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* S = sm;                        // dk x NS
     float* U = S + (size_t)dk * NS;       // C x NS
-    float* Wc = U + (size_t)C * NS;       // C x dk
+    float* Upc = U + (size_t)C * NS;      // C x NS: U' slice
+    float* PUc = Upc + (size_t)C * NS;    // C x NS: PU' slice
+    float* Wc = PUc + (size_t)C * NS;     // C x dk
     float* Qc = Wc + (size_t)C * dk;      // C x dk
     float* Kc = Qc + (size_t)C * dk;      // C x dk
     float* gc = Kc + (size_t)C * dk;      // dk
+
+    InterF32 L{C, dk, dv};
+    const float* inter = static_cast<const float*>(p.inter);
+    auto block = [&](int c) { return inter + ((size_t)bh * p.NC + c) * L.floats(); };
+    auto fetch_uo = [&](int c) {          // group: what the U / output phase reads
+        if (c < p.NC) {
+            const float* in = block(c);
+            cp_async_floats(Wc, in + L.W(), C * dk, tid);
+            cp_async_floats(Qc, in + L.Qe(), C * dk, tid);
+            cp_async_slice(Upc, in + L.Up() + j0, C, dv, tid);
+            cp_async_slice(PUc, in + L.PUp() + j0, C, dv, tid);
+        }
+        cp_async_commit_group();
+    };
+    auto fetch_s = [&](int c) {           // group: what the state update reads
+        if (c < p.NC) {
+            const float* in = block(c);
+            cp_async_floats(Kc, in + L.Kp(), C * dk, tid);
+            cp_async_floats(gc, in + L.gC(), dk, tid);
+        }
+        cp_async_commit_group();
+    };
 
     for (int idx = tid; idx < dk * NS; idx += kSimtThreads) {
         const int i = idx / NS, j = idx % NS;
         S[idx] = p.S0 ? p.S0[((size_t)bh * dk + i) * dv + j0 + j] : 0.f;
     }
-    InterF32 L{C, dk, dv};
+    fetch_uo(0);
+    fetch_s(0);
     Tout* out = static_cast<Tout*>(p.out);
     for (int c = 0; c < p.NC; ++c) {
-        const float* in = static_cast<const float*>(p.inter) + ((size_t)bh * p.NC + c) * L.floats();
-        __syncthreads();   // previous chunk's S update and U reads are done
+        cp_async_wait_one();              // W, Qe, U', PU' of chunk c
+        __syncthreads();                  // ... for every thread; S of chunk c is complete
         if (p.S_chunks) {
             float* dst = p.S_chunks + ((size_t)bh * p.NC + c) * dk * dv;
             for (int idx = tid; idx < dk * NS; idx += kSimtThreads) {
@@ -225,37 +279,67 @@ scan_simt_kernel(Problem p) {
                 dst[(size_t)i * dv + j0 + j] = S[idx];
             }
         }
-        for (int idx = tid; idx < C * dk; idx += kSimtThreads) {
-            Wc[idx] = in[L.W() + idx];
-            Qc[idx] = in[L.Qe() + idx];
-            Kc[idx] = in[L.Kp() + idx];
-        }
-        for (int i = tid; i < dk; i += kSimtThreads) gc[i] = in[L.gC() + i];
-        __syncthreads();
         const int s0 = c * C;
-        for (int idx = tid; idx < C * NS; idx += kSimtThreads) {
-            const int r = idx / NS, j = idx % NS;
-            float ws = 0.f, qs = 0.f;
-            for (int i = 0; i < dk; ++i) {
-                const float sij = S[(size_t)i * NS + j];
-                ws += Wc[(size_t)r * dk + i] * sij;
-                qs += Qc[(size_t)r * dk + i] * sij;
+        {   // thread: column j, rows rg, rg + 8, ...; each S[i][j] is read once for all its rows
+            const int j = tid % NS, rg = tid / NS;
+            float ws[NR], qs[NR];
+#pragma unroll
+            for (int m = 0; m < NR; ++m) { ws[m] = 0.f; qs[m] = 0.f; }
+            if (out) {
+                for (int i = 0; i < dk; ++i) {
+                    const float sij = S[(size_t)i * NS + j];
+#pragma unroll
+                    for (int m = 0; m < NR; ++m) {
+                        const int r = rg + kRowGroups * m;
+                        ws[m] += Wc[(size_t)r * dk + i] * sij;
+                        qs[m] += Qc[(size_t)r * dk + i] * sij;
+                    }
+                }
+            } else {                      // state recompute only: no outputs
+                for (int i = 0; i < dk; ++i) {
+                    const float sij = S[(size_t)i * NS + j];
+#pragma unroll
+                    for (int m = 0; m < NR; ++m) ws[m] += Wc[(size_t)(rg + kRowGroups * m) * dk + i] * sij;
+                }
             }
-            U[idx] = in[L.Up() + (size_t)r * dv + j0 + j] - ws;
-            const int s = s0 + r;
-            if (out && s < p.L) {     // no outputs in the backward's state recompute
-                RowRef rr = row_ref(p, b, h, s);
-                if (rr.has_q) store_out(out, rr.tok * dv + j0 + j, in[L.PUp() + (size_t)r * dv + j0 + j] + qs);
+#pragma unroll
+            for (int m = 0; m < NR; ++m) {
+                {
+                    const int r = rg + kRowGroups * m;
+                    const int idx = r * NS + j;
+                    U[idx] = Upc[idx] - ws[m];
+                    const int s = s0 + r;
+                    if (out && s < p.L) {
+                        RowRef rr = row_ref(p, b, h, s);
+                        if (rr.has_q) store_out(out, rr.tok * dv + j0 + j, PUc[idx] + qs[m]);
+                    }
+                }
             }
         }
+        __syncthreads();                  // W, Qe, U', PU' buffers are free; U is complete
+        fetch_uo(c + 1);
+        cp_async_wait_one();              // K', e^{g_C} of chunk c
         __syncthreads();
-        for (int idx = tid; idx < dk * NS; idx += kSimtThreads) {
-            const int i = idx / NS, j = idx % NS;
-            float acc = gc[i] * S[idx];
-            for (int r = 0; r < C; ++r) acc += Kc[(size_t)r * dk + i] * U[(size_t)r * NS + j];
-            S[idx] = acc;
+        {   // thread: column j, state rows ig, ig + 8, ...; each U[r][j] is read once
+            const int j = tid % NS, ig = tid / NS;
+            float acc[NI];
+#pragma unroll
+            for (int m = 0; m < NI; ++m) {
+                const int i = ig + kRowGroups * m;
+                acc[m] = gc[i] * S[(size_t)i * NS + j];
+            }
+            for (int r = 0; r < C; ++r) {
+                const float u = U[(size_t)r * NS + j];
+#pragma unroll
+                for (int m = 0; m < NI; ++m) acc[m] += Kc[(size_t)r * dk + ig + kRowGroups * m] * u;
+            }
+#pragma unroll
+            for (int m = 0; m < NI; ++m) S[(size_t)(ig + kRowGroups * m) * NS + j] = acc[m];
         }
+        __syncthreads();                  // K', e^{g_C} buffers are free
+        fetch_s(c + 1);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (p.S_final) {
         for (int idx = tid; idx < dk * NS; idx += kSimtThreads) {
@@ -275,6 +359,33 @@ bool simt_supported(int C, int dk, int dv) {
            dv % kScanCols == 0;
 }
 
+template <typename Tout, int NR, int NI>
+cudaError_t launch_scan_nr_ni(const Problem& p, dim3 grid, size_t smem, cudaStream_t stream) {
+    cudaFuncSetAttribute(scan_simt_kernel<Tout, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    scan_simt_kernel<Tout, NR, NI><<<grid, kSimtThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tout, int NR>
+cudaError_t launch_scan_nr(const Problem& p, dim3 grid, size_t smem, cudaStream_t stream) {
+    switch (p.dk / kRowGroups) {
+        case 4: return launch_scan_nr_ni<Tout, NR, 4>(p, grid, smem, stream);
+        case 8: return launch_scan_nr_ni<Tout, NR, 8>(p, grid, smem, stream);
+        case 16: return launch_scan_nr_ni<Tout, NR, 16>(p, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename Tout>
+cudaError_t launch_scan_t(const Problem& p, dim3 grid, size_t smem, cudaStream_t stream) {
+    switch (p.C / kRowGroups) {
+        case 2: return launch_scan_nr<Tout, 2>(p, grid, smem, stream);
+        case 4: return launch_scan_nr<Tout, 4>(p, grid, smem, stream);
+        case 8: return launch_scan_nr<Tout, 8>(p, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
     const size_t s1 = intra_simt_smem(p.C, p.dk, p.dv);
     const size_t s2 = scan_simt_smem(p.C, p.dk);
@@ -291,14 +402,7 @@ cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
     }
     dim3 g2(p.dv / kScanCols, p.B * p.H);
-    if (bf16) {
-        cudaFuncSetAttribute(scan_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
-        scan_simt_kernel<__nv_bfloat16><<<g2, kSimtThreads, s2, stream>>>(p);
-    } else {
-        cudaFuncSetAttribute(scan_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
-        scan_simt_kernel<float><<<g2, kSimtThreads, s2, stream>>>(p);
-    }
-    return cudaGetLastError();
+    return bf16 ? launch_scan_t<__nv_bfloat16>(p, g2, s2, stream) : launch_scan_t<float>(p, g2, s2, stream);
 }
 
 }  // namespace gdn
