@@ -22,7 +22,16 @@ Contents and what pins each part (the pins live in tests/test_oracle_*.py):
   spectral.*         closed forms (spectral norm of I - eta j k^T, the GDN2
                      shrink, the secular equation); pinned against numpy SVD /
                      eigenvalues on small matrices.
+  backward.gdn_grads gradients of the forward by fp64 autograd through the token
+                     loop; pinned by finite differences of the C forward and a
+                     one-token closed form (tests/test_oracle_backward_pins.py).
+  gdn2.*             GDN2 (non-tied erase / write) with the token-wise stability
+                     transforms, token by token and in non-tied WY chunks; pinned
+                     by the KDA case through gdn_seq, brute-force SVD of every
+                     transformed transition, and the two algorithms' agreement
+                     (tests/test_oracle_gdn2_pins.py).
 """
 from ._lib import build, deltaproduct_seq, gdn_seq, max_threads  # noqa: F401
 from .chunked import gdn_chunked  # noqa: F401
 from . import spectral  # noqa: F401
+from . import gdn2  # noqa: F401
