@@ -8,6 +8,7 @@ namespace gdn {
 // gdn_simt.cu
 size_t simt_inter_bytes(const Problem& p);
 bool simt_supported(int C, int dk, int dv);
+size_t simt_intra_smem_bytes(int C, int dk, int dv, bool gdn2);
 cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream);
 // gdn_tc.cu
 bool tc_supported(const Problem& p, bool bf16);
@@ -178,6 +179,52 @@ gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
     p.q = q; p.k = k; p.v = v; p.alpha = gamma; p.beta = beta;
     p.S0 = S0; p.out = out; p.S_final = S_final;
     return run(p, dtype == GDN_BF16, workspace, workspace_bytes, stream);
+}
+
+size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                     gdn_dtype_t dtype, unsigned flags) {
+    Problem p;
+    if (flags & ~(unsigned)GDN_ALPHA_SCALAR) return 0;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return 0;
+    if (simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return 0;
+    return kHeaderBytes + simt_inter_bytes(p);
+}
+
+int gdn2_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                            unsigned flags) {
+    if (gdn2_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype, flags) == 0) return -1;
+    if (B == 0 || H == 0) return 0;
+    return T > 0 ? 2 : 1;
+}
+
+gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* eta, const float* b_gate, const float* S0, void* out,
+                            float* S_final, int B, int H, int T, int dk, int dv, int chunk,
+                            gdn_dtype_t dtype, unsigned flags, int mode,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    if (flags & ~(unsigned)GDN_ALPHA_SCALAR) return GDN_ERR_INVALID_ARG;
+    if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
+    gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
+    if (st != GDN_OK) return st;
+    if (simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
+    const bool has_tokens = B > 0 && H > 0 && T > 0;
+    if (has_tokens && (!q || !k || !v || !alpha || !eta || !b_gate || !out)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, alpha, eta, b_gate, S0, out, S_final};
+    for (const void* x : ptrs)
+        if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
+    const size_t need = kHeaderBytes + simt_inter_bytes(p);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+        return GDN_ERR_WORKSPACE;
+    if (B == 0 || H == 0) return GDN_OK;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = nullptr;
+    p.S0 = S0; p.out = out; p.S_final = S_final;
+    p.gdn2_eta = eta ? eta : alpha;      // non-null marks GDN2 (eta is only read for T > 0)
+    p.gdn2_b = b_gate;
+    p.gdn2_mode = mode;
+    p.status = static_cast<int*>(workspace);
+    p.inter = static_cast<char*>(workspace) + kHeaderBytes;
+    return launch_simt(p, dtype == GDN_BF16, stream) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 size_t gdn_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,

@@ -13,9 +13,16 @@ constexpr int kRowGroups = kSimtThreads / kScanCols;   // 8: threads per column 
 // The scan kernel is instantiated per (chunk rows, state rows) a thread carries:
 // NR = C / 8 and NI = dk / 8, so its unrolled loops carry no idle iterations.
 
-// Shared memory of the intra kernel: qh, kt, g (C x dk), vt, Up (C x dv), A, Tm, P (C x C).
-__host__ __device__ inline size_t intra_simt_smem(int C, int dk, int dv) {
-    return sizeof(float) * ((size_t)3 * C * dk + (size_t)2 * C * dv + (size_t)3 * C * C);
+// Shared memory of the intra kernel: qh, kt, g (C x dk), vt, Up (C x dv), A, Tm, P (C x C),
+// and for GDN2 the erase vectors (C x dk).
+__host__ __device__ inline size_t intra_simt_smem(int C, int dk, int dv, bool gdn2 = false) {
+    return sizeof(float) * ((size_t)(gdn2 ? 4 : 3) * C * dk + (size_t)2 * C * dv + (size_t)3 * C * C);
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
 }
 
 // One CTA per (chunk, head).
@@ -40,6 +47,9 @@ intra_simt_kernel(Problem p) {
     float* A = Up + (size_t)C * dv;      // strictly lower A
     float* Tm = A + (size_t)C * C;       // T = (I + A)^{-1}
     float* P = Tm + (size_t)C * C;       // lower P
+    const bool gdn2 = p.gdn2_eta != nullptr;
+    // erase vectors: the rows A and the state read use (j' for GDN2; k~ itself otherwise)
+    float* ew = gdn2 ? P + (size_t)C * C : kt;
 
     const Tin* q = static_cast<const Tin*>(p.q);
     const Tin* k = static_cast<const Tin*>(p.k);
@@ -78,18 +88,50 @@ intra_simt_kernel(Problem p) {
             const bool bs = p.dp || p.beta_scalar;
             const bool as = p.dp || p.alpha_scalar;
             for (int j = lane; j < dk; j += 32) {
-                float bj = bs ? bscal : p.beta[rr.tok * dk + j];
+                float bj = gdn2 ? 1.f : (bs ? bscal : p.beta[rr.tok * dk + j]);
                 qr[j] *= iq;
                 kr[j] *= ik * sqrtf(bj);
                 gr[j] = as ? ascal : logf(p.alpha[rr.tok * dk + j]);
             }
-            for (int j = lane; j < dv; j += 32) {
-                float bj;
-                if (p.beta_v) bj = bs ? p.beta_v[rr.tok] : p.beta_v[rr.tok * dv + j];
-                else bj = bs ? bscal : p.beta[rr.tok * dk + j];   // channel-wise beta needs dk == dv
-                vr[j] = load_in(v, krow * dv + j) * sqrtf(bj);
+            if (gdn2) {
+                // GDN2 (Su Jianlin's GDN2 stability note, in the d_k x d_v convention): write
+                // vector k^, erase vector j' = eta k^ (.) b after the token-wise transform,
+                // values eta v.  kr already holds k^ (beta is not used).
+                const float eta = p.gdn2_eta[rr.tok];
+                float* er = ew + (size_t)r * dk;
+                float cdot = 0.f, nj2 = 0.f, amax = 0.f;
+                for (int j = lane; j < dk; j += 32) {
+                    kr[j] = load_in(k, krow * dk + j) * ik;
+                    const float jp = eta * kr[j] * p.gdn2_b[rr.tok * dk + j];
+                    er[j] = jp;
+                    cdot += jp * kr[j];
+                    nj2 += jp * jp;
+                    amax = fmaxf(amax, p.alpha_scalar ? p.alpha[rr.tok] : p.alpha[rr.tok * dk + j]);
+                }
+                cdot = warp_sum(cdot);
+                nj2 = warp_sum(nj2);
+                amax = warp_max(amax);
+                if (p.gdn2_mode == 1) {          // D -> min(D, 1/rho), rho = ||I - j' k^T||_2
+                    const float rho = 0.5f * (sqrtf(nj2) + sqrtf(fmaxf(nj2 - 4.f * cdot + 4.f, 0.f)));
+                    const float lr = -logf(rho);
+                    for (int j = lane; j < dk; j += 32) gr[j] = fminf(gr[j], lr);
+                } else if (p.gdn2_mode == 2) {   // j* = c k + lambda* (j' - c k)
+                    const float tau = (cdot - 1.f) * amax + 1.f / amax;
+                    const float den = nj2 - cdot * cdot;
+                    const float lam = den > 0.f ? fminf(1.f, sqrtf(fmaxf(tau * tau - cdot * cdot, 0.f) / den)) : 1.f;
+                    for (int j = lane; j < dk; j += 32) er[j] = cdot * kr[j] + lam * (er[j] - cdot * kr[j]);
+                }
+                for (int j = lane; j < dv; j += 32) vr[j] = load_in(v, krow * dv + j) * eta;
+            } else {
+                for (int j = lane; j < dv; j += 32) {
+                    float bj;
+                    if (p.beta_v) bj = bs ? p.beta_v[rr.tok] : p.beta_v[rr.tok * dv + j];
+                    else bj = bs ? bscal : p.beta[rr.tok * dk + j];   // channel-wise beta needs dk == dv
+                    vr[j] = load_in(v, krow * dv + j) * sqrtf(bj);
+                }
             }
         } else {
+            if (gdn2) for (int j = lane; j < dk; j += 32) ew[(size_t)r * dk + j] = 0.f;
             for (int j = lane; j < dk; j += 32) { qr[j] = 0.f; kr[j] = 0.f; gr[j] = 0.f; }
             for (int j = lane; j < dv; j += 32) vr[j] = 0.f;
         }
@@ -115,7 +157,7 @@ intra_simt_kernel(Problem p) {
                 const float e = expf(g[(size_t)r * dk + j] - g[(size_t)i * dk + j]);
                 const float ke = kt[(size_t)i * dk + j] * e;
                 pp += qh[(size_t)r * dk + j] * ke;
-                a += kt[(size_t)r * dk + j] * ke;
+                a += ew[(size_t)r * dk + j] * ke;
             }
             a = warp_sum(a);
             pp = warp_sum(pp);
@@ -150,7 +192,7 @@ intra_simt_kernel(Problem p) {
         const float gr = g[idx];
         outp[L.Kp() + idx] = kt[idx] * expf(gl - gr);
         const float eg = expf(gr);
-        kt[idx] *= eg;
+        ew[idx] *= eg;            // the state read: k~ e^g (tied) or j' e^g (GDN2)
         qh[idx] *= eg;
         (void)r;
     }
@@ -161,7 +203,7 @@ intra_simt_kernel(Problem p) {
     for (int idx = tid; idx < C * dk; idx += kSimtThreads) {
         const int r = idx / dk, j = idx % dk;
         float acc = 0.f;
-        for (int i = 0; i <= r; ++i) acc += Tm[(size_t)r * C + i] * kt[(size_t)i * dk + j];
+        for (int i = 0; i <= r; ++i) acc += Tm[(size_t)r * C + i] * ew[(size_t)i * dk + j];
         W[idx] = acc;
         outp[L.W() + idx] = acc;
     }
@@ -354,6 +396,8 @@ size_t simt_inter_bytes(const Problem& p) {
     return (size_t)p.B * p.H * p.NC * L.floats() * sizeof(float);
 }
 
+size_t simt_intra_smem_bytes(int C, int dk, int dv, bool gdn2) { return intra_simt_smem(C, dk, dv, gdn2); }
+
 bool simt_supported(int C, int dk, int dv) {
     return intra_simt_smem(C, dk, dv) <= 227 * 1024 && scan_simt_smem(C, dk) <= 227 * 1024 &&
            dv % kScanCols == 0;
@@ -387,7 +431,7 @@ cudaError_t launch_scan_t(const Problem& p, dim3 grid, size_t smem, cudaStream_t
 }
 
 cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
-    const size_t s1 = intra_simt_smem(p.C, p.dk, p.dv);
+    const size_t s1 = intra_simt_smem(p.C, p.dk, p.dv, p.gdn2_eta != nullptr);
     const size_t s2 = scan_simt_smem(p.C, p.dk);
     if (p.NC > 0) {
         dim3 g1(p.NC, p.B * p.H);

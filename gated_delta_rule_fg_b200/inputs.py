@@ -14,6 +14,8 @@ S0; DeltaProduct: q, k, v, beta, gamma-logits):
   S0       = 0, or ~ N(0, std 0.01)
   beta_v   = sigmoid(x), x ~ N(0, std)      (FG^2-GDN+ only; drawn last, after S0,
                                              [B,T,H,dv], or [B,T,H] with scalar beta)
+GDN2 (make_gdn2_inputs): q, k, v ~ N(0,1); alpha as above; eta = 2 sigmoid(N(0,1)) in
+  (0, 2); b = sigmoid(N(0, 2)) in (0, 1); S0 ~ N(0, s0_std); drawn in that order.
   DeltaProduct: beta ~ U[0, 2] per sub-step, gamma = sigmoid(x), x ~ N(2, 1)
 bf16 tensors are rounded to nearest-even from the float32 draws; the float32
 copy kept alongside holds exactly the rounded values.
@@ -132,3 +134,20 @@ def make_inputs(cfg: GdnConfig, *, seed: int | None = None, T: int | None = None
         vshape = (B, T, H) if cfg.beta_scalar else (B, T, H, cfg.dv)
         x["beta_v"] = _sigmoid(cfg.beta_std * rng.standard_normal(vshape, dtype=f32)).astype(f32)
     return x
+
+
+def make_gdn2_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype: str = "f32", seed: int = 0,
+                     alpha_scale: float = 0.1, s0_std: float = 0.1) -> dict:
+    """Seeded inputs of the GDN2 operator: q k v alpha eta b S0 (float32 numpy arrays
+    holding the stored values; q, k, v rounded to bf16 when dtype == "bf16")."""
+    rng = np.random.default_rng(seed)
+    rb = round_bf16 if dtype == "bf16" else (lambda a: a)
+    f32 = np.float32
+    q = rb(rng.standard_normal((B, T, H, dk), dtype=f32))
+    k = rb(rng.standard_normal((B, T, H, dk), dtype=f32))
+    v = rb(rng.standard_normal((B, T, H, dv), dtype=f32))
+    alpha = np.exp(-alpha_scale * _softplus(rng.standard_normal((B, T, H, dk), dtype=f32))).astype(f32)
+    eta = (2.0 * _sigmoid(rng.standard_normal((B, T, H), dtype=f32))).astype(f32)
+    b = _sigmoid(2.0 * rng.standard_normal((B, T, H, dk), dtype=f32)).astype(f32)
+    S0 = (s0_std * rng.standard_normal((B, H, dk, dv), dtype=f32)).astype(f32) if s0_std > 0 else None
+    return dict(q=q, k=k, v=v, alpha=alpha, eta=eta, b=b, S0=S0)

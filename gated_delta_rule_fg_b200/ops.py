@@ -44,6 +44,9 @@ SIGNATURES = {
     "gdn_chunk_bwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_chunk_bwd": (_I, [_P] * 16 + [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint, _P, _SZ, _P]),
     "gdn_chunk_bwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
+    "gdn2_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
+    "gdn2_chunk_fwd": (_I, [_P] * 9 + [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint, _I, _P, _SZ, _P]),
+    "gdn2_chunk_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_workspace_status": (_I, [_P, _P]),
     "gdn_status_string": (ctypes.c_char_p, [_I]),
     "gdn_version": (_I, []),
@@ -294,6 +297,43 @@ def chunk_bwd(q, k, v, alpha, beta, S0, dout, dS_final=None, *, beta_v=None, chu
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_bwd")
     return g
+
+
+GDN2_NONE, GDN2_CLIP_DECAY, GDN2_SHRINK_J = 0, 1, 2
+
+
+def gdn2_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:
+    return int(lib().gdn2_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags))
+
+
+def gdn2_chunk_fwd(q, k, v, alpha, eta, b_gate, S0=None, *, mode=GDN2_NONE, chunk=32,
+                   alpha_scalar=False, out=None, S_final=None, want_state=True, workspace=None,
+                   stream=None):
+    """GDN2 (non-tied erase j' = eta k^ (.) b, write k^) through gdn2_chunk_fwd, with the
+    token-wise stability transform `mode` (GDN2_NONE / GDN2_CLIP_DECAY / GDN2_SHRINK_J).
+    q, k [B,T,H,dk], v [B,T,H,dv]; alpha float32 [B,T,H,dk] (or [B,T,H]); eta float32
+    [B,T,H]; b_gate float32 [B,T,H,dk]; S0 float32 [B,H,dk,dv] or None."""
+    code = _dtype_code(q)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q.dtype)
+    for t, n in ((alpha, "alpha"), (eta, "eta"), (b_gate, "b_gate"), (S0, "S0")):
+        _check(t, n, torch.float32)
+    flags = GDN_ALPHA_SCALAR if alpha_scalar else 0
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    need = gdn2_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, code, flags)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    st = lib().gdn2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(eta), _ptr(b_gate), _ptr(S0),
+                              _ptr(out), _ptr(S_final), B, H, T, dk, dv, chunk, code, flags, int(mode),
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn2_chunk_fwd")
+    return out, S_final
 
 
 def recurrent_step(q, k, v, alpha, beta_k, S_in=None, *, beta_v=None, alpha_scalar=False,

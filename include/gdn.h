@@ -184,6 +184,44 @@ int gdn_plus_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, 
 int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
                                   gdn_dtype_t dtype);
 
+/* GDN2 transform modes (Su Jianlin's GDN2 stability note): none; clip the decay to
+ * min(D, 1/rho) with rho the closed-form spectral norm of I - j' k^T ("Simple
+ * Strategy"); or shrink j' toward KDA keeping j'^T k ("Modifying Itself"). */
+enum { GDN2_NONE = 0, GDN2_CLIP_DECAY = 1, GDN2_SHRINK_J = 2 };
+
+/* Bytes of workspace gdn2_chunk_fwd needs (0 if invalid/unsupported). */
+size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
+                                     gdn_dtype_t dtype, unsigned flags);
+
+/* GDN2 chunkwise forward: the non-tied update of Su Jianlin's GDN2 stability note
+ * ("Problem Description"), written for this library's d_k x d_v state X = S^T:
+ *     X_t = (I - k^_t j'_t^T) D_t X_{t-1} + eta_t k^_t v_t^T,    o_t = X_t^T q^_t
+ * with q^, k^ L2-normalised as above, j'_t = eta_t k^_t (.) b_t (GDN2's own
+ * parameterisation j = k (.) b, b in [0,1]^{dk}, with eta absorbed into j), and D_t =
+ * Diag(alpha_t) -- after the token-wise transform `mode` (GDN2_*): GDN2_CLIP_DECAY
+ * replaces D by min(D, 1/rho), rho = (||j'|| + sqrt(||j'||^2 - 4 j'^T k^ + 4)) / 2;
+ * GDN2_SHRINK_J replaces j' by c k^ + lambda* (j' - c k^), c = j'^T k^,
+ * tau = (c - 1) gamma_max + 1/gamma_max (gamma_max = max_i D_ii),
+ * lambda* = min(1, sqrt((tau^2 - c^2) / (||j'||^2 - c^2))).  With b = 1 and mode
+ * GDN2_NONE this is KDA with write rate eta.  The transforms are fused into the
+ * chunk's prep; the chunk form is the non-tied WY form (A pairs erase with write
+ * vectors, the state is read along j' and written along k^).
+ *   q, k [B,T,H,dk], v, out [B,T,H,dv]: dtype storage; alpha float32 [B,T,H,dk] (or
+ *   [B,T,H] with GDN_ALPHA_SCALAR, the only flag); eta float32 [B,T,H] (>= 0);
+ *   b_gate float32 [B,T,H,dk] in [0,1]; S0, S_final float32 [B,H,dk,dv] (may be NULL).
+ * Runs on the float32 CUDA-core path for both dtypes; chunk in {16, 32} (64 only
+ * where it fits shared memory), dk, dv in {32, 64, 128}.  Workspace and errors as
+ * gdn_chunk_fwd. */
+gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* eta, const float* b_gate, const float* S0, void* out,
+                            float* S_final, int B, int H, int T, int dk, int dv, int chunk,
+                            gdn_dtype_t dtype, unsigned flags, int mode,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of kernels one gdn2_chunk_fwd call enqueues (-1 if invalid/unsupported). */
+int gdn2_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                            unsigned flags);
+
 /* Bytes of workspace gdn_chunk_bwd needs (0 if invalid/unsupported). */
 size_t gdn_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
                                     gdn_dtype_t dtype, unsigned flags);

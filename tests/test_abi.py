@@ -166,3 +166,19 @@ def test_backward_validation(L):
     assert call(chunk=64) == ops.GDN_ERR_UNSUPPORTED
     assert call(ws=None) == ops.GDN_ERR_WORKSPACE
     assert call(dout=FAKE_ODD) == ops.GDN_ERR_INVALID_ARG
+
+
+def test_gdn2_validation(L):
+    ws = ops.gdn2_chunk_fwd_workspace_size
+    assert ws(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) > 0
+    assert ws(1, 2, 100, 128, 128, 64, ops.GDN_BF16, 0) == 0          # chunk 64 at d 128 does not fit
+    assert ws(1, 2, 100, 64, 64, 32, ops.GDN_F32, ops.GDN_BETA_SCALAR) == 0
+    assert L.gdn2_chunk_fwd_launches(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) == 2
+
+    def call(eta=FAKE, mode=0, chunk=32):
+        return L.gdn2_chunk_fwd(FAKE, FAKE, FAKE, FAKE, eta, FAKE, None, FAKE, None, 1, 1, 8, 64, 64, chunk,
+                                ops.GDN_F32, 0, mode, FAKE, 1 << 30, None)
+
+    assert call(eta=None) == ops.GDN_ERR_INVALID_ARG
+    assert call(mode=3) == ops.GDN_ERR_INVALID_ARG
+    assert call(chunk=48) == ops.GDN_ERR_UNSUPPORTED
