@@ -20,6 +20,8 @@
 // registers (one d_k row per thread); its fp16 copy is the MMA operand.
 // A producer warp streams the per-chunk blocks with bulk async copies into a
 // two-stage buffer.
+#include <mutex>
+
 #include "gdn_common.cuh"
 #include "gdn_sm100.cuh"
 
@@ -68,7 +70,9 @@ constexpr uint32_t kGlast = 111616;      // g_last [128]
 constexpr uint32_t kBar = 112128;        // mbarrier (MMA completion)
 constexpr uint32_t kBarK = 112144;       // mbarrier (K' reload)
 constexpr uint32_t kTmem = 112136;       // TMEM base address
-constexpr uint32_t kIntraSmem = 112192;
+constexpr uint32_t kEgr = 112192;        // e^{g_ref} [128]
+constexpr uint32_t kIntraSmem = 112704;
+static_assert(2 * (kIntraSmem + 1024) <= 228 * 1024, "two intra CTAs per SM (1 KB reserved each)");
 
 constexpr uint32_t kTmemCols = 256;
 // TMEM columns: D0 / D3 at 0, D1 (W~^T) at 64, D2 (U'^T) at 128, D4 (PU'^T) at 192.
@@ -112,9 +116,9 @@ __device__ __forceinline__ void record_timeout(int* status) {
 // ============================================================================ intra
 // kPlus: FG^2-GDN+ (separate value rate beta^v, eq. (13)).
 template <bool kPlus>
-__global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
+__global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     extern __shared__ __align__(1024) uint8_t sm[];
-    const int c = blockIdx.x;
+    const int c = cb + blockIdx.x;             // this launch covers chunks cb .. cb + gridDim.x - 1
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int s0 = c * C;
@@ -163,16 +167,21 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     // later overwrites with its own QG and KG octets; they are the first commit group, so
     // the norms wait for them alone.  (Holding them in registers through the norm and
     // prefix phases costs 32 registers and forces spills.)
-    if (!kPlus) {
+    // With beta^v (which takes the R0 slots), raw k goes to this thread's R1 slots (later
+    // its KIG octets) and only q stays in registers.
+    {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int o = o0 + 4 * j;
-            uint8_t* kdst = sm + kR0 + off_kmajor(r, 8 * o, 2048, 128);
-            uint8_t* qdst = sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128);
+            uint8_t* kdst = kPlus ? sm + kR1 + off_kmajor(r, 8 * o, 2048, 128)
+                                  : sm + kR0 + off_kmajor(r, 8 * o, 2048, 128);
             if (valid) cp_async16(kdst, k + krow * D + 8 * o);
             else *reinterpret_cast<uint4*>(kdst) = make_uint4(0, 0, 0, 0);
-            if (valid && rr.has_q) cp_async16(qdst, q + rr.tok * D + 8 * o);
-            else *reinterpret_cast<uint4*>(qdst) = make_uint4(0, 0, 0, 0);
+            if (!kPlus) {
+                uint8_t* qdst = sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128);
+                if (valid && rr.has_q) cp_async16(qdst, q + rr.tok * D + 8 * o);
+                else *reinterpret_cast<uint4*>(qdst) = make_uint4(0, 0, 0, 0);
+            }
         }
         cp_async_commit();
     }
@@ -200,10 +209,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
-        if (kPlus) {
-            qp[j] = (valid && rr.has_q) ? ldg16(q + rr.tok * D + 8 * o) : make_uint4(0, 0, 0, 0);
-            kp[j] = valid ? ldg16(k + krow * D + 8 * o) : make_uint4(0, 0, 0, 0);
-        }
+        if (kPlus) qp[j] = (valid && rr.has_q) ? ldg16(q + rr.tok * D + 8 * o) : make_uint4(0, 0, 0, 0);
         if (valid && !a_scalar) {
             al0[j] = ldg16f(p.alpha + rr.tok * D + 8 * o);
             al1[j] = ldg16f(p.alpha + rr.tok * D + 8 * o + 4);
@@ -212,16 +218,14 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             al1[j] = al0[j];
         }
     }
-    if (!kPlus) cp_async_wait_group<1>();      // q and k (the older group) have landed
+    cp_async_wait_group<1>();      // raw k (and q without beta^v), the older group, has landed
     float ssq = 0.f, ssk = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
         float fq[8], fk[8];
-        if (!kPlus) {
-            qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
-            kp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
-        }
+        if (!kPlus) qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
+        kp[j] = *reinterpret_cast<const uint4*>(sm + (kPlus ? kR1 : kR0) + off_kmajor(r, 8 * o, 2048, 128));
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
 #pragma unroll
@@ -292,6 +296,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         const float gr = fallback ? 0.f : 0.5f * glast[tid];
         gref[tid] = gr;
         fK[tid] = __expf(glast[tid] - gr);
+        reinterpret_cast<float*>(sm + kEgr)[tid] = __expf(gr);
         reinterpret_cast<float*>(blk + kOffGC)[tid] = __expf(glast[tid]);
     }
     __syncthreads();
@@ -307,7 +312,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     {
         const long nxt = (long)blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
         if (p.prefetch_ahead > 0 && nxt < (long)gridDim.x * gridDim.y) {
-            const int c2 = (int)(nxt % gridDim.x), bh2 = (int)(nxt / gridDim.x);
+            const int c2 = cb + (int)(nxt % gridDim.x), bh2 = (int)(nxt / gridDim.x);
             const int r2 = tid >> 2, part = tid & 3;        // 4 threads per row
             const int s2 = c2 * C + r2;
             if (s2 < p.L) {
@@ -359,10 +364,9 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         }
         const uint4 vp = valid ? *reinterpret_cast<const uint4*>(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128))
                                : make_uint4(0, 0, 0, 0);
-        if (!kPlus) {      // reread from shared memory: not held in registers across the phases
-            qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
-            kp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
-        }
+        // reread from shared memory: not held in registers across the phases
+        if (!kPlus) qp[j] = *reinterpret_cast<const uint4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
+        kp[j] = *reinterpret_cast<const uint4*>(sm + (kPlus ? kR1 : kR0) + off_kmajor(r, 8 * o, 2048, 128));
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
         bf8_to_f(vp, fv);
@@ -638,7 +642,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
     tc_fence_after();
     if (ok && warp < 4) {        // Qe -> block (MN-major (r, c)); PU' -> block (fp16, sw rows)
         const int ch = 32 * warp + lane;
-        const float er = __expf(gref[ch]);
+        const float er = reinterpret_cast<const float*>(sm + kEgr)[ch];
         const uint32_t lanebase = t0 + ((uint32_t)(32 * warp) << 16);
         float x0[32], x1[32];
         tmem_ld32(lanebase + 0, x0);
@@ -653,9 +657,16 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
         }
         tmem_ld32(lanebase + 192, x0);
         tmem_ld32(lanebase + 224, x1);
-        __half* pu = reinterpret_cast<__half*>(blk + kOffPU) + (size_t)(ch / NS) * C * NS;
+        // Warp w holds PU' slice w (its 32 channels, all rows): build the slice's block image
+        // in the dead T32 area (R6), then copy it out as 16-byte vectors.
+        __half* st = reinterpret_cast<__half*>(sm + kR6 + warp * (C * NS * 2));
 #pragma unroll
-        for (int r2 = 0; r2 < C; ++r2) pu[sw_half(r2, ch % NS)] = __float2half_rn(r2 < 32 ? x0[r2] : x1[r2 - 32]);
+        for (int r2 = 0; r2 < C; ++r2) st[sw_half(r2, lane)] = __float2half_rn(r2 < 32 ? x0[r2] : x1[r2 - 32]);
+        __syncwarp();
+        const uint4* srcv = reinterpret_cast<const uint4*>(st);
+        uint4* dstv = reinterpret_cast<uint4*>(blk + kOffPU + warp * (C * NS * 2));
+#pragma unroll
+        for (int i = 0; i < C * NS * 2 / 16 / 32; ++i) dstv[lane + 32 * i] = srcv[lane + 32 * i];
     } else if (ok) {             // N = N~ * e^{g_ref[c]} (column scale) -> block (K-major (i, c))
         const int row = 32 * (warp & 3) + lane;
         const uint32_t lanebase = t0 + ((uint32_t)(32 * (warp & 3)) << 16);
@@ -664,7 +675,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p) {
             float x[32];
             tmem_ld32(lanebase + 64 + c0, x);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] *= __expf(gref[c0 + e]);
+            for (int e = 0; e < 32; ++e) x[e] *= reinterpret_cast<const float*>(sm + kEgr)[c0 + e];
 #pragma unroll
             for (int g8 = 0; g8 < 32; g8 += 8)
                 *reinterpret_cast<uint4*>(blk + kOffN + off_kmajor(row, c0 + g8, 2048, 128)) = f_to_h8(x + g8);
@@ -735,7 +746,10 @@ constexpr uint32_t kSBar = kSop + 3 * 8192;                // 230912: mbarriers
 constexpr uint32_t kSTmem = kSBar + 256;
 constexpr uint32_t kScanSmem = kSTmem + 64;                // 231232
 
-__global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
+// This launch covers chunks cb .. ce-1, starting from S_in (null: zero) and leaving the
+// state in S_out (may be null); ring stages and barrier phases count from cb.
+__global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int cb, int ce,
+                                                                  const float* S_in, float* S_out) {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int slice = blockIdx.x;
     const int bh = blockIdx.y;
@@ -751,6 +765,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
     uint64_t* o_free = s_ready + 1;        // [2] D_O buffer read (4 warp arrivals)
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kSTmem);
     const uint8_t* blocks = static_cast<const uint8_t*>(p.inter) + (size_t)bh * p.NC * kBlockBytes;
+    const int nloc = ce - cb;              // chunks of this launch; loop indices below are local
 
     if (warp == 0) {
         tmem_alloc(tslot, 128);
@@ -777,8 +792,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
     if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            for (int ch = 0; ch < p.NC && ok; ++ch) {
-                const uint8_t* src = blocks + (size_t)ch * kBlockBytes;
+            for (int ch = 0; ch < nloc && ok; ++ch) {
+                const uint8_t* src = blocks + (size_t)(cb + ch) * kBlockBytes;
                 const int s3 = ch % kNB, s4 = ch % kQP;
                 if (ch >= kNB && !mbar_wait(&emptyNB[s3], ((ch / kNB) - 1) & 1)) { ok = false; break; }
                 uint8_t* d3 = sm + kRingNB + s3 * kNBStride;
@@ -812,7 +827,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
                 mma_commit(&bar_o[cc & 1]);
                 return true;
             };
-            for (int ch = 0; ch < p.NC && ok; ++ch) {
+            for (int ch = 0; ch < nloc && ok; ++ch) {
                 const int s3 = ch % kNB;
                 if (!mbar_wait(s_ready, ch & 1) || !mbar_wait(&fullNB[s3], (ch / kNB) & 1)) { ok = false; break; }
                 tc_fence_after();
@@ -825,7 +840,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
                 }
                 if (ch > 0 && !issue_o(ch - 1)) { ok = false; break; }
             }
-            if (ok && p.NC > 0) ok = issue_o(p.NC - 1);
+            if (ok && nloc > 0) ok = issue_o(nloc - 1);
             if (!ok) record_timeout(p.status);
         }
     } else if (warp < 4) {
@@ -835,13 +850,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
         const uint32_t lanebase = (uint32_t)(32 * warp) << 16;
         float S[NS];
 #pragma unroll
-        for (int j = 0; j < NS; ++j) S[j] = p.S0 ? p.S0[((size_t)bh * D + row) * D + j0 + j] : 0.f;
+        for (int j = 0; j < NS; ++j) S[j] = S_in ? S_in[((size_t)bh * D + row) * D + j0 + j] : 0.f;
 #pragma unroll
         for (int j = 0; j < NS; j += 8) st16(sm + kSop, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_ready);
-        for (int ch = 0; ch < p.NC && ok; ++ch) {
+        for (int ch = 0; ch < nloc && ok; ++ch) {
             const int s3 = ch % kNB;
             const uint8_t* nb = sm + kRingNB + s3 * kNBStride;
             if (!__all_sync(0xffffffffu, mbar_wait(&fullNB[s3], (ch / kNB) & 1))) { ok = false; break; }
@@ -878,8 +893,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
         }
         if (!ok) {
             if (lane == 0) record_timeout(p.status);
-        } else if (p.S_final) {
-            float4* dst = reinterpret_cast<float4*>(p.S_final + ((size_t)bh * D + row) * D + j0);
+        } else if (S_out) {
+            float4* dst = reinterpret_cast<float4*>(S_out + ((size_t)bh * D + row) * D + j0);
 #pragma unroll
             for (int j = 0; j < NS; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
@@ -890,7 +905,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
         const uint32_t lanebase = (uint32_t)(32 * wq) << 16;
         const int rw = 16 * wq + lane;                         // output row (valid for lane < 16)
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-        for (int ch = 0; ch < p.NC && ok; ++ch) {
+        for (int ch = 0; ch < nloc && ok; ++ch) {
             const int s4 = ch % kQP;
             const bool got = mbar_wait(&fullQP[s4], (ch / kQP) & 1) && mbar_wait(&bar_o[ch & 1], (ch >> 1) & 1);
             if (!__all_sync(0xffffffffu, got)) {
@@ -904,7 +919,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[ch & 1]);
             if (lane < 16) {
-                const int s = ch * C + rw;
+                const int s = (cb + ch) * C + rw;
                 if (s < p.L) {
                     const RowRef ro = row_ref(p, b, h, s);
                     if (ro.has_q) {
@@ -941,16 +956,63 @@ bool tc_supported(const Problem& p, bool bf16) {
     return bf16 && p.C == tc::C && p.dk == tc::D && p.dv == tc::D && p.T > 0;
 }
 
-size_t tc_inter_bytes(const Problem& p) { return (size_t)p.B * p.H * p.NC * tc::kBlockBytes; }
+// Segments of one call: the sequence's chunks are cut into P consecutive ranges.  Intra of
+// range s+1 runs on the caller's stream while the scan of range s runs on a high-priority
+// side stream, so the scan's chain no longer waits for the whole intra role and the SMs
+// the scan leaves idle keep working.  Each range keeps at least kMinSegChunks chunks.
+constexpr int kMaxSegments = 4;
+constexpr int kMinSegChunks = 32;
 
-int tc_launches(const Problem& p) { return p.NC > 0 ? 2 : 1; }
+int tc_segments(const Problem& p) {
+    const int s = p.NC / kMinSegChunks;
+    return s < 1 ? 1 : (s > kMaxSegments ? kMaxSegments : s);
+}
+
+size_t tc_inter_bytes(const Problem& p) {
+    const size_t blocks = (size_t)p.B * p.H * p.NC * tc::kBlockBytes;   // 256-byte multiple
+    const size_t handoff = tc_segments(p) > 1 ? (size_t)p.B * p.H * tc::D * tc::D * sizeof(float) : 0;
+    return blocks + handoff;
+}
+
+int tc_launches(const Problem& p) { return p.NC > 0 ? 2 * tc_segments(p) : 1; }
+
+namespace {
+
+// Per device: the side stream and the fork / per-range / join events, created on first use.
+// One mutex covers the creation and every enqueue sequence that uses them.
+struct SideStream {
+    bool tried = false, ok = false;
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, ready[kMaxSegments] = {};
+};
+constexpr int kMaxDev = 64;
+SideStream g_side[kMaxDev];
+std::mutex g_side_mu;
+
+bool side_stream_ready(SideStream& ss) {
+    if (ss.tried) return ss.ok;
+    ss.tried = true;
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return false;
+    if (cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi) != cudaSuccess) return false;
+    bool ok = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kMaxSegments && ok; ++i)
+        ok = cudaEventCreateWithFlags(&ss.ready[i], cudaEventDisableTiming) == cudaSuccess;
+    ss.ok = ok;
+    return ok;
+}
+
+}  // namespace
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>;
     cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+    cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
     Problem pi = p;
+    int dev = 0;
     {
-        int dev = 0, sms = 0, per_sm = 0;
+        int sms = 0, per_sm = 0;
         if (cudaGetDevice(&dev) == cudaSuccess &&
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra, tc::NT, tc::kIntraSmem) == cudaSuccess)
@@ -958,14 +1020,37 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
         else
             pi.prefetch_ahead = 0;
     }
-    cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
-    dim3 g1(p.NC, p.B * p.H);
-    intra<<<g1, tc::NT, tc::kIntraSmem, stream>>>(pi);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    dim3 g2(tc::J, p.B * p.H);
-    tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, stream>>>(p);
-    return cudaGetLastError();
+    const dim3 g2(tc::J, p.B * p.H);
+    const int P = tc_segments(p);
+    if (P == 1 || dev < 0 || dev >= kMaxDev) {
+        intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, 0);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
+        return cudaGetLastError();
+    }
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream& ss = g_side[dev];
+    if (!side_stream_ready(ss)) return cudaErrorUnknown;
+    float* handoff = reinterpret_cast<float*>(static_cast<char*>(p.inter) +
+                                              (size_t)p.B * p.H * p.NC * tc::kBlockBytes);
+    cudaError_t e = cudaEventRecord(ss.fork, stream);             // the side stream starts after
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.fork, 0);   // the caller's prior work
+    for (int sg = 0; sg < P && e == cudaSuccess; ++sg) {
+        const int cb = (int)((long)p.NC * sg / P), ce = (int)((long)p.NC * (sg + 1) / P);
+        intra<<<dim3(ce - cb, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, cb);
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.ready[sg], 0);
+        if (e != cudaSuccess) break;
+        tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, ss.stream>>>(
+            p, cb, ce, sg == 0 ? p.S0 : handoff, sg == P - 1 ? p.S_final : handoff);
+        e = cudaGetLastError();
+    }
+    // join: whatever happened above, the caller's stream waits for the side stream's work
+    cudaError_t j = cudaEventRecord(ss.join, ss.stream);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(stream, ss.join, 0);
+    return e != cudaSuccess ? e : j;
 }
 
 }  // namespace gdn

@@ -44,7 +44,14 @@
  *     `workspace` (device memory, 256-byte aligned, at least the size the
  *     matching *_workspace_size function returns); one workspace must not be
  *     used by two calls that can run at the same time.  The library allocates
- *     nothing and keeps no global state.
+ *     no device memory.  For long sequences on the tensor-core path it keeps,
+ *     per device and created on first use, one high-priority stream and a few
+ *     events: a call then forks onto that stream (so part of its work overlaps)
+ *     and joins back before returning, so all of its work is still ordered
+ *     after earlier and before later work on `stream`, and stream capture
+ *     records the fork and the join.  Enqueuing such calls from several host
+ *     threads on one device serialises on a lock; capturing one while another
+ *     thread enqueues on the same device is not supported.
  *   - Arguments are validated before anything is enqueued; on an error
  *     nothing is enqueued.  Errors found on the device (a bounded wait that
  *     ran out, a value outside the fp16 operand range) are recorded in the

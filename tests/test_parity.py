@@ -233,3 +233,12 @@ def test_plus_full_size_sampled_heads():
     x = make_inputs(cfg)
     pairs = [(0, 0), (0, cfg.H - 1)]
     check(cfg, run_plus(cfg, x), oracle_plus(cfg, x, pairs=pairs), pairs=pairs)
+
+
+def test_tensor_core_segmented_call_uneven_ranges():
+    """A sequence long enough for the call to be cut into chunk ranges whose intra and scan
+    roles overlap on two streams (98 chunks: three uneven ranges) with a ragged last chunk
+    and a nonzero initial state: every token and the final state match the oracle."""
+    cfg = GdnConfig("tcseg", B=1, H=2, T=64 * 97 + 13, dk=128, dv=128, chunk=64, s0_std=0.05, seed=6100)
+    x = make_inputs(cfg)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
