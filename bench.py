@@ -276,6 +276,29 @@ def build_op(args, cfg, ops, torch, dev, stream, rank):
                   abytes=B * H * per_head, flops=float(B * H * 6 * cfg.dk * cfg.dv), tokens=B,
                   metric=f"tokens/s FG²-GDN decode step (B={B} sequences, H={H}, d={cfg.dk}), 1 B200",
                   e2e_in=["q", "k", "v", "alpha", "beta"], e2e_out=[o], kernel="gdn_recurrent_step")
+    if op == "gdn2":
+        from gated_delta_rule_fg_b200.inputs import make_gdn2_inputs
+        chunk = 32
+        g = make_gdn2_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, dtype=cfg.dtype, seed=cfg.seed + 1000 * rank)
+        dg = {k: (torch.from_numpy(v).to(dev) if v is not None else None) for k, v in g.items()}
+        for kname in ("q", "k", "v"):
+            dg[kname] = dg[kname].to(dt)
+        out = torch.empty((B, T, H, cfg.dv), dtype=dt, device=dev)
+        Sf = torch.empty((B, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
+        nws = ops.gdn2_chunk_fwd_workspace_size(B, H, T, cfg.dk, cfg.dv, chunk, code, 0)
+        ws = ops.alloc_workspace(nws, dev)
+
+        def step(src):
+            ops.gdn2_chunk_fwd(src["q"], src["k"], src["v"], src["alpha"], src["eta"], src["b"], src["S0"],
+                               mode=ops.GDN2_CLIP_DECAY, chunk=chunk, out=out, S_final=Sf, workspace=ws,
+                               stream=stream)
+        per = (2 * cfg.dk + 2 * cfg.dv) * e + 2 * cfg.dk * 4 + 4
+        return Op(cfg=cfg, d=dg, host=None, step=step, ws=ws,
+                  launches=int(ops.lib().gdn2_chunk_fwd_launches(B, H, T, cfg.dk, cfg.dv, chunk, code, 0)),
+                  abytes=th * per + B * H * cfg.dk * cfg.dv * 4 * 2, flops=algorithmic_flops(cfg), tokens=B * T,
+                  metric=f"tokens/s GDN2 chunked fwd with the decay clip (T={T}, d={cfg.dk}, chunk {chunk}, "
+                         f"float32 path), 1 B200",
+                  e2e_in=None, e2e_out=None, kernel="gdn2_chunk_fwd")
     if op == "bwd":
         chunk = 16
         nws = ops.chunk_bwd_workspace_size(B, H, T, cfg.dk, cfg.dv, chunk, code, flags)
@@ -333,9 +356,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="fg2_prefill_32k", choices=sorted(CONFIGS))
-    ap.add_argument("--op", default="fwd", choices=["fwd", "plus", "decode", "bwd"],
+    ap.add_argument("--op", default="fwd", choices=["fwd", "plus", "decode", "bwd", "gdn2"],
                     help="fwd: the chunked forward (the headline); plus: FG²-GDN+ forward; decode: one "
-                         "recurrent step per sequence (B=256 by default); bwd: the chunked backward")
+                         "recurrent step per sequence (B=256 by default); bwd: the chunked backward; "
+                         "gdn2: GDN2 with the decay clip (float32 path)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

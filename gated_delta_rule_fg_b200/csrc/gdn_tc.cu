@@ -968,6 +968,22 @@ int tc_segments(const Problem& p) {
     return s < 1 ? 1 : (s > kMaxSegments ? kMaxSegments : s);
 }
 
+// Chunk range [cb, ce) of segment sg of P.  Only the last range's scan runs with no intra
+// work beside it, and a chunk's intra role costs several times its scan step, so the last
+// range is short (NC/8, at least kMinSegChunks) and the others share the rest evenly.
+void seg_range(int NC, int P, int sg, int& cb, int& ce) {
+    int last = NC / 8 > kMinSegChunks ? NC / 8 : kMinSegChunks;
+    if (last > NC / P) last = NC / P;
+    const int head = NC - last;
+    if (sg == P - 1) {
+        cb = head;
+        ce = NC;
+    } else {
+        cb = (int)((long)head * sg / (P - 1));
+        ce = (int)((long)head * (sg + 1) / (P - 1));
+    }
+}
+
 size_t tc_inter_bytes(const Problem& p) {
     const size_t blocks = (size_t)p.B * p.H * p.NC * tc::kBlockBytes;   // 256-byte multiple
     const size_t handoff = tc_segments(p) > 1 ? (size_t)p.B * p.H * tc::D * tc::D * sizeof(float) : 0;
@@ -1037,7 +1053,8 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     cudaError_t e = cudaEventRecord(ss.fork, stream);             // the side stream starts after
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.fork, 0);   // the caller's prior work
     for (int sg = 0; sg < P && e == cudaSuccess; ++sg) {
-        const int cb = (int)((long)p.NC * sg / P), ce = (int)((long)p.NC * (sg + 1) / P);
+        int cb, ce;
+        seg_range(p.NC, P, sg, cb, ce);
         intra<<<dim3(ce - cb, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, cb);
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
