@@ -278,7 +278,7 @@ def build_op(args, cfg, ops, torch, dev, stream, rank):
                   e2e_in=["q", "k", "v", "alpha", "beta"], e2e_out=[o], kernel="gdn_recurrent_step")
     if op == "gdn2":
         from gated_delta_rule_fg_b200.inputs import make_gdn2_inputs
-        chunk = 32
+        chunk = cfg.chunk
         g = make_gdn2_inputs(cfg.B, cfg.T, cfg.H, cfg.dk, cfg.dv, dtype=cfg.dtype, seed=cfg.seed + 1000 * rank)
         dg = {k: (torch.from_numpy(v).to(dev) if v is not None else None) for k, v in g.items()}
         for kname in ("q", "k", "v"):
@@ -296,8 +296,8 @@ def build_op(args, cfg, ops, torch, dev, stream, rank):
         return Op(cfg=cfg, d=dg, host=None, step=step, ws=ws,
                   launches=int(ops.lib().gdn2_chunk_fwd_launches(B, H, T, cfg.dk, cfg.dv, chunk, code, 0)),
                   abytes=th * per + B * H * cfg.dk * cfg.dv * 4 * 2, flops=algorithmic_flops(cfg), tokens=B * T,
-                  metric=f"tokens/s GDN2 chunked fwd with the decay clip (T={T}, d={cfg.dk}, chunk {chunk}, "
-                         f"float32 path), 1 B200",
+                  metric=f"tokens/s GDN2 chunked fwd with the decay clip (T={T}, d={cfg.dk}, chunk {chunk}), "
+                         f"1 B200",
                   e2e_in=None, e2e_out=None, kernel="gdn2_chunk_fwd")
     if op == "bwd":
         chunk = 16
@@ -359,7 +359,7 @@ def main():
     ap.add_argument("--op", default="fwd", choices=["fwd", "plus", "decode", "bwd", "gdn2"],
                     help="fwd: the chunked forward (the headline); plus: FG²-GDN+ forward; decode: one "
                          "recurrent step per sequence (B=256 by default); bwd: the chunked backward; "
-                         "gdn2: GDN2 with the decay clip (float32 path)")
+                         "gdn2: GDN2 with the decay clip")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--ref-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

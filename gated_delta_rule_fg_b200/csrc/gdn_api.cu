@@ -186,6 +186,7 @@ size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int ch
     Problem p;
     if (flags & ~(unsigned)GDN_ALPHA_SCALAR) return 0;
     if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return 0;
+    if (tc_supported(p, dtype == GDN_BF16)) return kHeaderBytes + tc_inter_bytes(p);
     if (simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return 0;
     return kHeaderBytes + simt_inter_bytes(p);
 }
@@ -194,6 +195,9 @@ int gdn2_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_
                             unsigned flags) {
     if (gdn2_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype, flags) == 0) return -1;
     if (B == 0 || H == 0) return 0;
+    Problem p;
+    make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
+    if (tc_supported(p, dtype == GDN_BF16)) return tc_launches(p);
     return T > 0 ? 2 : 1;
 }
 
@@ -207,13 +211,14 @@ gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const f
     if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
     gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
     if (st != GDN_OK) return st;
-    if (simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
+    const bool tc = tc_supported(p, dtype == GDN_BF16);
+    if (!tc && simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return GDN_ERR_UNSUPPORTED;
     const bool has_tokens = B > 0 && H > 0 && T > 0;
     if (has_tokens && (!q || !k || !v || !alpha || !eta || !b_gate || !out)) return GDN_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, alpha, eta, b_gate, S0, out, S_final};
     for (const void* x : ptrs)
         if (!aligned16(x)) return GDN_ERR_INVALID_ARG;
-    const size_t need = kHeaderBytes + simt_inter_bytes(p);
+    const size_t need = kHeaderBytes + (tc ? tc_inter_bytes(p) : simt_inter_bytes(p));
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return GDN_ERR_WORKSPACE;
     if (B == 0 || H == 0) return GDN_OK;
@@ -224,7 +229,8 @@ gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const f
     p.gdn2_mode = mode;
     p.status = static_cast<int*>(workspace);
     p.inter = static_cast<char*>(workspace) + kHeaderBytes;
-    return launch_simt(p, dtype == GDN_BF16, stream) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    const cudaError_t e = tc ? launch_tc(p, stream) : launch_simt(p, dtype == GDN_BF16, stream);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 size_t gdn_chunk_bwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,

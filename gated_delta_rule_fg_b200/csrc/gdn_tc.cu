@@ -115,7 +115,10 @@ __device__ __forceinline__ void record_timeout(int* status) {
 
 // ============================================================================ intra
 // kPlus: FG^2-GDN+ (separate value rate beta^v, eq. (13)).
-template <bool kPlus>
+// kG2: GDN2 (Su Jianlin's GDN2 stability note): the A rows and the state read use the erase
+// vector j' = eta k^ (.) b after the token-wise transform, the write vector is k^, and v is
+// scaled by eta; everything after the prep is the tied computation.
+template <bool kPlus, bool kG2 = false>
 __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     extern __shared__ __align__(1024) uint8_t sm[];
     const int c = cb + blockIdx.x;             // this launch covers chunks cb .. cb + gridDim.x - 1
@@ -189,10 +192,11 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int o = o0 + 4 * j;
-            if (!b_scalar) {
+            if (!b_scalar) {      // beta, or GDN2's gate b (always channel-wise)
+                const float* bsrc = kG2 ? p.gdn2_b : p.beta;
                 float* dst = bstage + (r * 16 + (o ^ (r & 7))) * 8;
-                cp_async16(dst, p.beta + rr.tok * D + 8 * o);
-                cp_async16(dst + 4, p.beta + rr.tok * D + 8 * o + 4);
+                cp_async16(dst, bsrc + rr.tok * D + 8 * o);
+                cp_async16(dst + 4, bsrc + rr.tok * D + 8 * o + 4);
             }
             cp_async16(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128), v + krow * D + 8 * o);
             if (kPlus && !b_scalar) {
@@ -252,6 +256,49 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             if (kPlus && p.beta_scalar) bv_s = p.beta_v[rr.tok];
         }
     }
+    // GDN2 row quantities: c = j'^T k^, ||j'||^2 and max alpha over the row's 4 lanes, then
+    // the transform: the clip bound on log alpha (mode 1) or the shrink factor (mode 2).
+    float g2_eta = 0.f, g2_c = 0.f, g2_lam = 1.f, g2_lr = 0.f;
+    if constexpr (kG2) {
+        cp_async_wait_all();       // the gate b has landed (this thread's own slots)
+        float cd = 0.f, nj = 0.f, am = 0.f;
+        if (valid) {
+            g2_eta = p.gdn2_eta[rr.tok];
+            const float as_ = a_scalar ? p.alpha[rr.tok] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int o = o0 + 4 * j;
+                const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+                float fk[8];
+                bf8_to_f(kp[j], fk);
+                const float a8[8] = {al0[j].x, al0[j].y, al0[j].z, al0[j].w, al1[j].x, al1[j].y, al1[j].z, al1[j].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float kh = fk[e] * ik;
+                    const float jp = g2_eta * kh * bsrc[e];
+                    cd += jp * kh;
+                    nj += jp * jp;
+                    am = fmaxf(am, a_scalar ? as_ : a8[e]);
+                }
+            }
+        }
+        cd += __shfl_xor_sync(0xffffffffu, cd, 8);
+        cd += __shfl_xor_sync(0xffffffffu, cd, 16);
+        nj += __shfl_xor_sync(0xffffffffu, nj, 8);
+        nj += __shfl_xor_sync(0xffffffffu, nj, 16);
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 8));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 16));
+        g2_c = cd;
+        if (valid && p.gdn2_mode == 1) {          // D -> min(D, 1/rho)
+            const float rho = 0.5f * (sqrtf(nj) + sqrtf(fmaxf(nj - 4.f * cd + 4.f, 0.f)));
+            g2_lr = -__logf(rho);
+        }
+        if (valid && p.gdn2_mode == 2) {          // j* = c k + lambda* (j' - c k)
+            const float tau = (cd - 1.f) * am + 1.f / am;
+            const float den = nj - cd * cd;
+            g2_lam = den > 0.f ? fminf(1.f, sqrtf(fmaxf(tau * tau - cd * cd, 0.f) / den)) : 1.f;
+        }
+    }
     // log alpha, inclusive scan over the 8 rows of this warp (lanes with equal o0)
     float la[4][8];
 #pragma unroll
@@ -264,6 +311,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             const float4 a0 = al0[j], a1 = al1[j];
             la[j][0] = __logf(a0.x); la[j][1] = __logf(a0.y); la[j][2] = __logf(a0.z); la[j][3] = __logf(a0.w);
             la[j][4] = __logf(a1.x); la[j][5] = __logf(a1.y); la[j][6] = __logf(a1.z); la[j][7] = __logf(a1.w);
+        }
+        if (kG2 && valid && p.gdn2_mode == 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) la[j][e] = fminf(la[j][e], g2_lr);
         }
 #pragma unroll
         for (int d = 1; d < 8; d <<= 1) {
@@ -305,6 +356,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     float* fb_g = reinterpret_cast<float*>(blk + kOffB);                  // fallback scratch: g fp32 [C][D]
     __half* fb_k = reinterpret_cast<__half*>(blk + kOffPU);               // k~ fp16 [C][D]
     __half* fb_q = reinterpret_cast<__half*>(blk + kOffN);                // q^ fp16 [C][D]
+    __half* fb_e = fb_q + C * D;                                          // GDN2 erase fp16 [C][D]
     cp_async_wait_all();     // this thread's own staged beta and v
     // The CTAs of one wave load together and then compute with HBM idle.  Now that this
     // CTA's inputs have arrived, start the next wave's: the CTA prefetch_ahead places
@@ -325,8 +377,8 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
                     prefetch_l2(v + kr2 * D + 64 * part);
                 }
                 if (!a_scalar) prefetch_l2(p.alpha + rp.tok * D + 32 * part);
-                if (!b_scalar) {
-                    prefetch_l2(p.beta + rp.tok * D + 32 * part);
+                if (!b_scalar) {  // beta, or GDN2's gate b (p.beta is null there)
+                    prefetch_l2((kG2 ? p.gdn2_b : p.beta) + rp.tok * D + 32 * part);
                     if (kPlus) prefetch_l2(p.beta_v + rp.tok * D + 32 * part);
                 }
             }
@@ -335,10 +387,17 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
-        float g[8], sb[8], sv[8], fq[8], fk[8], fv[8];
+        float g[8], sb[8], sv[8], fq[8], fk[8], fv[8], gb[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) g[e] = la[j][e] + scr[warp * D + 8 * o + e];
-        if (b_scalar || !valid) {
+        if (kG2) {                // no beta: k~ = k^; the gate b feeds the erase vector
+            const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                sb[e] = valid ? 1.f : 0.f;
+                gb[e] = valid ? bsrc[e] : 0.f;
+            }
+        } else if (b_scalar || !valid) {
             const float s = valid ? sqrtf(b_s) : 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) sb[e] = s;
@@ -349,7 +408,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             sb[0] = sqrtf(b0.x); sb[1] = sqrtf(b0.y); sb[2] = sqrtf(b0.z); sb[3] = sqrtf(b0.w);
             sb[4] = sqrtf(b1.x); sb[5] = sqrtf(b1.y); sb[6] = sqrtf(b1.z); sb[7] = sqrtf(b1.w);
         }
-        if (!kPlus) {
+        if (kG2) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sv[e] = g2_eta;
+        } else if (!kPlus) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) sv[e] = sb[e];
         } else if (b_scalar || !valid) {
@@ -370,7 +432,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
         bf8_to_f(qp[j], fq);
         bf8_to_f(kp[j], fk);
         bf8_to_f(vp, fv);
-        float KG[8], QG[8], KIG[8], VT[8], KP[8], KT[8], QH[8];
+        float KG[8], QG[8], KIG[8], VT[8], KP[8], KT[8], QH[8], EJ[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             const int ch = 8 * o + e;
@@ -379,9 +441,16 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             const float exi = __expf(gr - g[e]);
             const float kt = fk[e] * ik * sb[e];
             const float qh = fq[e] * iq;
+            // the erase (A-row, state-read) vector: k~ itself, or GDN2's j' (shrunk in mode 2)
+            float er = kt;
+            if (kG2) {
+                const float jp = g2_eta * kt * gb[e];
+                er = g2_lam * jp + (1.f - g2_lam) * g2_c * kt;
+            }
+            EJ[e] = er;
             KT[e] = kt;
             QH[e] = qh;
-            KG[e] = kt * ex;
+            KG[e] = er * ex;
             QG[e] = qh * ex;
             KIG[e] = kt * exi;
             VT[e] = fv[e] * sv[e];
@@ -400,6 +469,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             for (int e = 0; e < 8; ++e) fb_g[r * D + 8 * o + e] = g[e];
             *reinterpret_cast<uint4*>(fb_k + r * D + 8 * o) = f_to_h8(KT);
             *reinterpret_cast<uint4*>(fb_q + r * D + 8 * o) = f_to_h8(QH);
+            if (kG2) *reinterpret_cast<uint4*>(fb_e + r * D + 8 * o) = f_to_h8(EJ);
         }
     }
     fence_async_smem();
@@ -439,7 +509,8 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             for (int i = 0; i < 32; ++i) acc[i] = 0.f;
             for (int ch = 0; ch < D; ++ch) {
                 const float gr = fb_g[rowr * D + ch];
-                const float xr = __half2float(isP ? fb_q[rowr * D + ch] : fb_k[rowr * D + ch]);
+                const float xr = __half2float(isP ? fb_q[rowr * D + ch]
+                                                  : (kG2 ? fb_e[rowr * D + ch] : fb_k[rowr * D + ch]));
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int col = cb + i;
@@ -1022,7 +1093,8 @@ bool side_stream_ready(SideStream& ss) {
 }  // namespace
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
-    auto intra = p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>;
+    auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
+               : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
     cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
     cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
     Problem pi = p;

@@ -216,9 +216,10 @@ size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int ch
  *   q, k [B,T,H,dk], v, out [B,T,H,dv]: dtype storage; alpha float32 [B,T,H,dk] (or
  *   [B,T,H] with GDN_ALPHA_SCALAR, the only flag); eta float32 [B,T,H] (>= 0);
  *   b_gate float32 [B,T,H,dk] in [0,1]; S0, S_final float32 [B,H,dk,dv] (may be NULL).
- * Runs on the float32 CUDA-core path for both dtypes; chunk in {16, 32} (64 only
- * where it fits shared memory), dk, dv in {32, 64, 128}.  Workspace and errors as
- * gdn_chunk_fwd. */
+ * GDN_BF16 with chunk 64 and dk == dv == 128 runs on the tensor-core path (fp16
+ * operands, as gdn_chunk_fwd); other shapes run on the float32 CUDA-core path with
+ * chunk in {16, 32} (64 only where it fits shared memory).  dk, dv in {32, 64, 128}.
+ * Workspace and errors as gdn_chunk_fwd. */
 gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const float* alpha,
                             const float* eta, const float* b_gate, const float* S0, void* out,
                             float* S_final, int B, int H, int T, int dk, int dv, int chunk,

@@ -112,7 +112,10 @@ def test_plus_validation(L):
     assert ops.chunk_fwd_workspace_size(1, 2, 100, 64, 128, 32, ops.GDN_F32, 0) == 0
     assert pws(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == \
         ops.chunk_fwd_workspace_size(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0)
-    assert ops.plus_chunk_fwd_launches(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == 2
+    # 512 chunks: four chunk ranges, each an intra and a scan launch
+    assert ops.plus_chunk_fwd_launches(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == 8
+    assert ops.chunk_fwd_launches(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == 8
+    assert ops.chunk_fwd_launches(1, 16, 2048, 128, 128, 64, ops.GDN_BF16, 0) == 2      # 32 chunks: one range
     assert pws(1, 1, 10, 96, 96, 64, ops.GDN_F32, 0) == 0
 
     def call(beta_v=FAKE, **kw):
@@ -171,7 +174,8 @@ def test_backward_validation(L):
 def test_gdn2_validation(L):
     ws = ops.gdn2_chunk_fwd_workspace_size
     assert ws(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) > 0
-    assert ws(1, 2, 100, 128, 128, 64, ops.GDN_BF16, 0) == 0          # chunk 64 at d 128 does not fit
+    assert ws(1, 2, 100, 128, 128, 64, ops.GDN_F32, 0) == 0           # float32 path: chunk 64 at d 128 does not fit
+    assert ws(1, 2, 100, 128, 128, 64, ops.GDN_BF16, 0) > 0           # ... the tensor-core path takes it
     assert ws(1, 2, 100, 64, 64, 32, ops.GDN_F32, ops.GDN_BETA_SCALAR) == 0
     assert L.gdn2_chunk_fwd_launches(1, 2, 100, 64, 64, 32, ops.GDN_F32, 0) == 2
 

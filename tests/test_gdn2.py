@@ -62,3 +62,31 @@ def test_gdn2_clip_keeps_state_bounded_where_plain_grows():
         parity(got[1], rs, TOL_F32)
         if mode == "clip":
             assert np.linalg.norm(got[1]) <= np.linalg.norm(x["S0"]) * (1 + 1e-4)
+
+
+TC = [(mode, T) for mode in MODES for T in (1, 63, 200)]
+
+
+@pytest.mark.parametrize("mode,T", TC)
+def test_gdn2_tensor_core(mode, T):
+    """bf16, chunk 64, d = 128 runs on the tensor-core kernels (erase operand in the A rows and
+    the state read); fp16 operands, so the bf16 bound of the tied path applies."""
+    from _util import TOL_BF16
+    x = make_gdn2_inputs(2, T, 2, 128, 128, dtype="bf16", seed=5300 + T + len(mode))
+    got = run(x, "bf16", 64, mode)
+    ro, rs = oracle_gdn2.gdn2_seq(x["q"], x["k"], x["v"], x["alpha"], x["eta"], x["b"], x["S0"], mode=mode)
+    parity(got[0], ro, TOL_BF16, out_bf16=True)
+    parity(got[1], rs, TOL_BF16)
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_gdn2_tensor_core_strong_decay_fallback(mode):
+    """Chunks with a wide log-decay span take the element-wise fp32 Gram products, which read
+    the erase rows the prep stored for them."""
+    from _util import TOL_BF16
+    x = make_gdn2_inputs(1, 200, 2, 128, 128, dtype="bf16", seed=5400 + len(mode))
+    x["alpha"] = np.where(np.arange(200)[None, :, None, None] % 3 == 0, 1e-6, x["alpha"]).astype(np.float32)
+    got = run(x, "bf16", 64, mode)
+    ro, rs = oracle_gdn2.gdn2_seq(x["q"], x["k"], x["v"], x["alpha"], x["eta"], x["b"], x["S0"], mode=mode)
+    parity(got[0], ro, TOL_BF16, out_bf16=True)
+    parity(got[1], rs, TOL_BF16)
