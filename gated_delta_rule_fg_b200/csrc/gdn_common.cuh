@@ -23,6 +23,8 @@
 // O = (Q^ (.) e^g) S + P U and the next state is Diag(e^{g_C}) S + K'^T U;
 // substituting U = U' - W S into O gives O = Qe S + PU'.
 #pragma once
+#include <mutex>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -106,5 +108,16 @@ struct InterF32 {
     __host__ __device__ size_t PUp() const { return 3 * (size_t)C * dk + (size_t)C * dv; }
     __host__ __device__ size_t gC() const { return 3 * (size_t)C * dk + 2 * (size_t)C * dv; }
 };
+
+// Per device: one high-priority stream and a few events, created on first use, onto which a
+// call forks part of its work (fork / join through events on the caller's stream).
+constexpr int kSideEvents = 8;
+struct SideStream {
+    cudaStream_t stream;
+    cudaEvent_t fork, join, ready[kSideEvents];
+};
+// Takes the side-stream lock (held by `lock` for the caller's whole enqueue sequence) and
+// returns the current device's side stream, or null if it cannot be created.
+SideStream* side_stream_lock(std::unique_lock<std::mutex>& lock);
 
 }  // namespace gdn

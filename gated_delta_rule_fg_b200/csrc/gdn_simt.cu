@@ -338,10 +338,14 @@ scan_simt_kernel(Problem p) {
                     }
                 }
             } else {                      // state recompute only: no outputs
-                for (int i = 0; i < dk; ++i) {
-                    const float sij = S[(size_t)i * NS + j];
+                for (int i = 0; i < dk; i += 4) {   // W rows as float4 along i
+                    const float s0 = S[(size_t)i * NS + j], s1 = S[(size_t)(i + 1) * NS + j];
+                    const float s2 = S[(size_t)(i + 2) * NS + j], s3 = S[(size_t)(i + 3) * NS + j];
 #pragma unroll
-                    for (int m = 0; m < NR; ++m) ws[m] += Wc[(size_t)(rg + kRowGroups * m) * dk + i] * sij;
+                    for (int m = 0; m < NR; ++m) {
+                        const float4 w = *reinterpret_cast<const float4*>(Wc + (size_t)(rg + kRowGroups * m) * dk + i);
+                        ws[m] += w.x * s0 + w.y * s1 + w.z * s2 + w.w * s3;
+                    }
                 }
             }
 #pragma unroll
@@ -362,21 +366,26 @@ scan_simt_kernel(Problem p) {
         fetch_uo(c + 1);
         cp_async_wait_one();              // K', e^{g_C} of chunk c
         __syncthreads();
-        {   // thread: column j, state rows ig, ig + 8, ...; each U[r][j] is read once
-            const int j = tid % NS, ig = tid / NS;
+        {   // thread: column j, state rows i0 .. i0 + NI - 1 (contiguous: K' rows load as
+            // float4); each U[r][j] is read once
+            const int j = tid % NS, i0 = (tid / NS) * NI;
             float acc[NI];
 #pragma unroll
-            for (int m = 0; m < NI; ++m) {
-                const int i = ig + kRowGroups * m;
-                acc[m] = gc[i] * S[(size_t)i * NS + j];
-            }
+            for (int m = 0; m < NI; ++m) acc[m] = gc[i0 + m] * S[(size_t)(i0 + m) * NS + j];
             for (int r = 0; r < C; ++r) {
                 const float u = U[(size_t)r * NS + j];
+                const float4* kv = reinterpret_cast<const float4*>(Kc + (size_t)r * dk + i0);
 #pragma unroll
-                for (int m = 0; m < NI; ++m) acc[m] += Kc[(size_t)r * dk + ig + kRowGroups * m] * u;
+                for (int m4 = 0; m4 < NI / 4; ++m4) {
+                    const float4 kk = kv[m4];
+                    acc[4 * m4 + 0] += kk.x * u;
+                    acc[4 * m4 + 1] += kk.y * u;
+                    acc[4 * m4 + 2] += kk.z * u;
+                    acc[4 * m4 + 3] += kk.w * u;
+                }
             }
 #pragma unroll
-            for (int m = 0; m < NI; ++m) S[(size_t)(ig + kRowGroups * m) * NS + j] = acc[m];
+            for (int m = 0; m < NI; ++m) S[(size_t)(i0 + m) * NS + j] = acc[m];
         }
         __syncthreads();                  // K', e^{g_C} buffers are free
         fetch_s(c + 1);
@@ -430,9 +439,8 @@ cudaError_t launch_scan_t(const Problem& p, dim3 grid, size_t smem, cudaStream_t
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
+cudaError_t launch_simt_intra(const Problem& p, bool bf16, cudaStream_t stream) {
     const size_t s1 = intra_simt_smem(p.C, p.dk, p.dv, p.gdn2_eta != nullptr);
-    const size_t s2 = scan_simt_smem(p.C, p.dk);
     if (p.NC > 0) {
         dim3 g1(p.NC, p.B * p.H);
         if (bf16) {
@@ -442,11 +450,20 @@ cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
             cudaFuncSetAttribute(intra_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
             intra_simt_kernel<float><<<g1, kSimtThreads, s1, stream>>>(p);
         }
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+        return cudaGetLastError();
     }
+    return cudaSuccess;
+}
+
+cudaError_t launch_simt_scan(const Problem& p, bool bf16, cudaStream_t stream) {
+    const size_t s2 = scan_simt_smem(p.C, p.dk);
     dim3 g2(p.dv / kScanCols, p.B * p.H);
     return bf16 ? launch_scan_t<__nv_bfloat16>(p, g2, s2, stream) : launch_scan_t<float>(p, g2, s2, stream);
+}
+
+cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream) {
+    cudaError_t e = launch_simt_intra(p, bf16, stream);
+    return e != cudaSuccess ? e : launch_simt_scan(p, bf16, stream);
 }
 
 }  // namespace gdn

@@ -1032,6 +1032,7 @@ bool tc_supported(const Problem& p, bool bf16) {
 // side stream, so the scan's chain no longer waits for the whole intra role and the SMs
 // the scan leaves idle keep working.  Each range keeps at least kMinSegChunks chunks.
 constexpr int kMaxSegments = 4;
+static_assert(kMaxSegments <= kSideEvents, "one ready event per range");
 constexpr int kMinSegChunks = 32;
 
 int tc_segments(const Problem& p) {
@@ -1063,34 +1064,6 @@ size_t tc_inter_bytes(const Problem& p) {
 
 int tc_launches(const Problem& p) { return p.NC > 0 ? 2 * tc_segments(p) : 1; }
 
-namespace {
-
-// Per device: the side stream and the fork / per-range / join events, created on first use.
-// One mutex covers the creation and every enqueue sequence that uses them.
-struct SideStream {
-    bool tried = false, ok = false;
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr, ready[kMaxSegments] = {};
-};
-constexpr int kMaxDev = 64;
-SideStream g_side[kMaxDev];
-std::mutex g_side_mu;
-
-bool side_stream_ready(SideStream& ss) {
-    if (ss.tried) return ss.ok;
-    ss.tried = true;
-    int lo = 0, hi = 0;
-    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return false;
-    if (cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, hi) != cudaSuccess) return false;
-    bool ok = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess &&
-              cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) == cudaSuccess;
-    for (int i = 0; i < kMaxSegments && ok; ++i)
-        ok = cudaEventCreateWithFlags(&ss.ready[i], cudaEventDisableTiming) == cudaSuccess;
-    ss.ok = ok;
-    return ok;
-}
-
-}  // namespace
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
@@ -1110,16 +1083,18 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     }
     const dim3 g2(tc::J, p.B * p.H);
     const int P = tc_segments(p);
-    if (P == 1 || dev < 0 || dev >= kMaxDev) {
+    auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream
         intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
         return cudaGetLastError();
-    }
-    std::lock_guard<std::mutex> lock(g_side_mu);
-    SideStream& ss = g_side[dev];
-    if (!side_stream_ready(ss)) return cudaErrorUnknown;
+    };
+    if (P == 1) return one_stream();
+    std::unique_lock<std::mutex> lock;
+    SideStream* side = side_stream_lock(lock);
+    if (!side) return one_stream();
+    SideStream& ss = *side;
     float* handoff = reinterpret_cast<float*>(static_cast<char*>(p.inter) +
                                               (size_t)p.B * p.H * p.NC * tc::kBlockBytes);
     cudaError_t e = cudaEventRecord(ss.fork, stream);             // the side stream starts after
