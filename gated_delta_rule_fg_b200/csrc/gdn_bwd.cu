@@ -34,7 +34,8 @@
 
 namespace gdn {
 
-cudaError_t launch_simt(const Problem& p, bool bf16, cudaStream_t stream);
+cudaError_t launch_simt_intra(const Problem& p, bool bf16, cudaStream_t stream);
+cudaError_t launch_simt_scan(const Problem& p, bool bf16, cudaStream_t stream);
 
 namespace bwd {
 
@@ -147,10 +148,14 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
             float acc[NR];
 #pragma unroll
             for (int m = 0; m < NR; ++m) acc[m] = 0.f;
-            for (int i = 0; i < dk; ++i) {
-                const float x = dS[(size_t)i * kNS + j];
+            for (int i = 0; i < dk; i += 4) {    // K' rows as float4 along i
+                const float x0 = dS[(size_t)i * kNS + j], x1 = dS[(size_t)(i + 1) * kNS + j];
+                const float x2 = dS[(size_t)(i + 2) * kNS + j], x3 = dS[(size_t)(i + 3) * kNS + j];
 #pragma unroll
-                for (int m = 0; m < NR; ++m) acc[m] += Kc[(size_t)(rg + kGroups * m) * dk + i] * x;
+                for (int m = 0; m < NR; ++m) {
+                    const float4 kk = *reinterpret_cast<const float4*>(Kc + (size_t)(rg + kGroups * m) * dk + i);
+                    acc[m] += kk.x * x0 + kk.y * x1 + kk.z * x2 + kk.w * x3;
+                }
             }
 #pragma unroll
             for (int m = 0; m < NR; ++m) Y[(size_t)(rg + kGroups * m) * kNS + j] = acc[m];
@@ -160,24 +165,27 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
         wait_all_but_newest();               // W, Qe, e^{g_C}, dO of chunk c
         __syncthreads();
         // dS <- Diag(gC) dS' - W^T Y + Qe^T dO   (element (i, j) reads only its own dS')
-        {   // thread: column j, state rows ig, ig + 8, ...; dO[r][j], Y[r][j] read once
-            const int j = tid % kNS, ig = tid / kNS;
+        {   // thread: column j, state rows i0 .. i0 + NI - 1 (contiguous, so the Qe and W rows
+            // load as float4); dO[r][j], Y[r][j] read once per r
+            const int j = tid % kNS, i0 = (tid / kNS) * NI;
             float acc[NI];
 #pragma unroll
-            for (int m = 0; m < NI; ++m) {
-                const int i = ig + kGroups * m;
-                acc[m] = gc[i] * dS[(size_t)i * kNS + j];
-            }
+            for (int m = 0; m < NI; ++m) acc[m] = gc[i0 + m] * dS[(size_t)(i0 + m) * kNS + j];
             for (int r = 0; r < C; ++r) {
                 const float d = load_in(dOs, (size_t)r * kNS + j), y = Y[(size_t)r * kNS + j];
+                const float4* qv = reinterpret_cast<const float4*>(Qc + (size_t)r * dk + i0);
+                const float4* wv = reinterpret_cast<const float4*>(Wc + (size_t)r * dk + i0);
 #pragma unroll
-                for (int m = 0; m < NI; ++m) {
-                    const int i = ig + kGroups * m;
-                    acc[m] += Qc[(size_t)r * dk + i] * d - Wc[(size_t)r * dk + i] * y;
+                for (int m4 = 0; m4 < NI / 4; ++m4) {
+                    const float4 qq = qv[m4], ww = wv[m4];
+                    acc[4 * m4 + 0] += qq.x * d - ww.x * y;
+                    acc[4 * m4 + 1] += qq.y * d - ww.y * y;
+                    acc[4 * m4 + 2] += qq.z * d - ww.z * y;
+                    acc[4 * m4 + 3] += qq.w * d - ww.w * y;
                 }
             }
 #pragma unroll
-            for (int m = 0; m < NI; ++m) dS[(size_t)(ig + kGroups * m) * kNS + j] = acc[m];
+            for (int m = 0; m < NI; ++m) dS[(size_t)(i0 + m) * kNS + j] = acc[m];
         }
         __syncthreads();                     // W, Qe, e^{g_C}, dO buffers free
         fetch_b(c - 1);
@@ -209,7 +217,7 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     constexpr int nwarps = NT / 32;
 
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* qh = sm;                          // q^                      C x dk
     float* kt = qh + (size_t)C * dk;         // k~
     float* g = kt + (size_t)C * dk;          // log alpha, then cumulative
@@ -325,9 +333,13 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
         for (int idx = tid; idx < C * kNS; idx += NT) {
             const int r = idx / kNS, jj = idx % kNS;
             float ks = 0.f, kd = 0.f;
-            for (int i = 0; i < dk; ++i) {
-                ks += KG[(size_t)r * dk + i] * St[i * kLd + jj];
-                kd += KE[(size_t)r * dk + i] * dSt[i * kLd + jj];
+            for (int i = 0; i < dk; i += 4) {    // K_G, K_E rows as float4 along i
+                const float4 g4 = *reinterpret_cast<const float4*>(KG + (size_t)r * dk + i);
+                const float4 e4 = *reinterpret_cast<const float4*>(KE + (size_t)r * dk + i);
+                ks += g4.x * St[i * kLd + jj] + g4.y * St[(i + 1) * kLd + jj] +
+                      g4.z * St[(i + 2) * kLd + jj] + g4.w * St[(i + 3) * kLd + jj];
+                kd += e4.x * dSt[i * kLd + jj] + e4.y * dSt[(i + 1) * kLd + jj] +
+                      e4.z * dSt[(i + 2) * kLd + jj] + e4.w * dSt[(i + 3) * kLd + jj];
             }
             U[(size_t)r * dv + jt + jj] = vt[(size_t)r * dv + jt + jj] - ks;
             dR[(size_t)r * dv + jt + jj] = kd;
@@ -390,15 +402,23 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
             dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
         }
         __syncthreads();
-        for (int jj = 0; jj < kNS; ++jj) {
-            const float s = St[cc * kLd + jj], ds = dSt[cc * kLd + jj];
-            if (r0 == 0) G4 += s * ds;
+        for (int jj = 0; jj < kNS; jj += 4) {   // four columns at a time: row data as float4
+            float sv[4], dv4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sv[e] = St[cc * kLd + jj + e];
+                dv4[e] = dSt[cc * kLd + jj + e];
+                if (r0 == 0) G4 += sv[e] * dv4[e];
+            }
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
                 const size_t o = (size_t)(r0 + rstep * m) * dv + jt + jj;
-                G1[m] += dOs[o] * s;
-                G2[m] += dR[o] * s;
-                G3[m] += U[o] * ds;
+                const float4 a = *reinterpret_cast<const float4*>(dOs + o);
+                const float4 rr4 = *reinterpret_cast<const float4*>(dR + o);
+                const float4 u = *reinterpret_cast<const float4*>(U + o);
+                G1[m] += a.x * sv[0] + a.y * sv[1] + a.z * sv[2] + a.w * sv[3];
+                G2[m] += rr4.x * sv[0] + rr4.y * sv[1] + rr4.z * sv[2] + rr4.w * sv[3];
+                G3[m] += u.x * dv4[0] + u.y * dv4[1] + u.z * dv4[2] + u.w * dv4[3];
             }
         }
     }
@@ -527,10 +547,13 @@ cudaError_t launch_grad(const Problem& p, const Grads& gr, cudaStream_t stream) 
 }
 
 template <typename Tin>
-cudaError_t launch_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
-    cudaError_t e = (p.C / kGroups == 2) ? launch_rev_nr<Tin, 2>(p, gr, stream)
-                  : (p.C / kGroups == 4) ? launch_rev_nr<Tin, 4>(p, gr, stream) : cudaErrorInvalidValue;
-    if (e != cudaSuccess || p.NC == 0) return e;
+cudaError_t launch_rev_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    return (p.C / kGroups == 2) ? launch_rev_nr<Tin, 2>(p, gr, stream)
+         : (p.C / kGroups == 4) ? launch_rev_nr<Tin, 4>(p, gr, stream) : cudaErrorInvalidValue;
+}
+
+template <typename Tin>
+cudaError_t launch_grad_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
     switch (p.C * p.dk / NT) {
         case 2: return launch_grad<Tin, 2>(p, gr, stream);
         case 4: return launch_grad<Tin, 4>(p, gr, stream);
@@ -566,14 +589,36 @@ cudaError_t launch_bwd(Problem p, const void* dO, const float* dS_final, float* 
     p.S_chunks = reinterpret_cast<float*>(base + up(fwd_inter));
     bwd::Grads gr{dO, dS_final, dq, dk, dv, dalpha, dbeta, dbeta_v, dS0,
                   reinterpret_cast<float*>(base + up(fwd_inter) + up(states))};
-    if (p.NC > 0) {
-        Problem f = p;                 // state recompute: no outputs, chunk-start states kept
-        f.out = nullptr;
-        f.S_final = nullptr;
-        cudaError_t e = launch_simt(f, bf16, stream);
-        if (e != cudaSuccess) return e;
+    auto rev = [&](cudaStream_t st) {
+        return bf16 ? bwd::launch_rev_t<__nv_bfloat16>(p, gr, st) : bwd::launch_rev_t<float>(p, gr, st);
+    };
+    if (p.NC == 0) return rev(stream);        // dS0 = dS_final
+    Problem f = p;                             // state recompute: no outputs, chunk-start states kept
+    f.out = nullptr;
+    f.S_final = nullptr;
+    cudaError_t e = launch_simt_intra(f, bf16, stream);
+    if (e != cudaSuccess) return e;
+    {
+        // The recompute scan (forward over chunks) and the state-gradient scan (backward over
+        // chunks) both read only the chunk blocks: run them side by side, the second on the
+        // side stream, and join before the gradient kernel.
+        std::unique_lock<std::mutex> lock;
+        SideStream* ss = side_stream_lock(lock);
+        if (!ss) {
+            e = launch_simt_scan(f, bf16, stream);
+            if (e == cudaSuccess) e = rev(stream);
+        } else {
+            e = cudaEventRecord(ss->fork, stream);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+            if (e == cudaSuccess) e = rev(ss->stream);
+            if (e == cudaSuccess) e = launch_simt_scan(f, bf16, stream);
+            cudaError_t j = cudaEventRecord(ss->join, ss->stream);
+            if (j == cudaSuccess) j = cudaStreamWaitEvent(stream, ss->join, 0);
+            if (e == cudaSuccess) e = j;
+        }
     }
-    return bf16 ? bwd::launch_t<__nv_bfloat16>(p, gr, stream) : bwd::launch_t<float>(p, gr, stream);
+    if (e != cudaSuccess) return e;
+    return bf16 ? bwd::launch_grad_t<__nv_bfloat16>(p, gr, stream) : bwd::launch_grad_t<float>(p, gr, stream);
 }
 
 }  // namespace gdn
