@@ -14,12 +14,20 @@
 // inputs of the later products; the per-channel factor e^{g_ref} is put back in
 // the epilogue.
 //
+// The intra kernel also forms N = -K'^T W and b = K'^T U', so the chunk update
+// S <- Diag(gC) S + K'^T (U' - W S) becomes S <- Diag(gC) S + N S + b: one
+// tensor-core product per chunk on the serial path.
+//
 // scan_tc_kernel: one CTA per (head, 32-column slice of d_v), serial over the
-// chunks.  Per chunk: D1 = [W; Qe] S (one M = 128 MMA), U = U' - D1[0:64],
-// O = PU' + D1[64:128]; D2 = K'^T U; S <- Diag(gC) S + D2.  S stays in fp32
-// registers (one d_k row per thread); its fp16 copy is the MMA operand.
-// A producer warp streams the per-chunk blocks with bulk async copies into a
-// two-stage buffer.
+// chunks of its range.  Per chunk: D_S = N S (M = 128, the chain), then
+// S <- Diag(gC) S + D_S + b in fp32 registers (one d_k row per thread; the fp16
+// copy is the next B operand); off the chain, D_O = Qe S (M = 64) and
+// O = D_O + PU'.  A producer warp streams the per-chunk blocks with bulk async
+// copies into two rings, one thread issues every MMA, and all hand-offs are
+// bounded mbarrier waits.
+//
+// launch_tc cuts long sequences into chunk ranges: intra of range s+1 runs on
+// the caller's stream while the scan of range s runs on the side stream.
 #include <mutex>
 
 #include "gdn_common.cuh"
