@@ -573,18 +573,19 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 
     // ---------------------------------------------------------------- T = (I + A)^{-1}
     // Blocked forward substitution in fp32: four 16x16 diagonal blocks in registers
-    // (lane j carries column j; row r of A is broadcast by shuffles), then
+    // (lane j carries column j; row r of A is a broadcast shared-memory read, which
+    // does not depend on the running solution and so issues ahead of it; fetching it
+    // from other lanes by shuffles ran as fast here but depended on how the compiler
+    // ordered the exchanges -- one instrumented build ran that loop ~15x slower), then
     // T10 = -T11 A10 T00 on 16x16 and 32x32 blocks.
     if (warp < 4) {
         const int bb = 16 * warp, jc = lane & 15;
-        float acol[16], t[16];
-#pragma unroll
-        for (int r2 = 0; r2 < 16; ++r2) acol[r2] = A32[sw64(bb + r2, bb + jc)];
+        float t[16];
 #pragma unroll
         for (int r2 = 0; r2 < 16; ++r2) {
             float acc = (r2 == jc) ? 1.f : 0.f;
 #pragma unroll
-            for (int i = 0; i < r2; ++i) acc -= __shfl_sync(0xffffffffu, acol[r2], i) * t[i];
+            for (int i = 0; i < r2; ++i) acc -= A32[sw64(bb + r2, bb + i)] * t[i];
             t[r2] = acc;
         }
         if (lane < 16) {
