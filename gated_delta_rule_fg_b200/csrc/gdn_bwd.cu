@@ -371,22 +371,47 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
         }
         __syncthreads();
     }
-    // 5. dP = lower(dO U^T), dA = strictly-lower(-dR U^T)
-    for (int pr = warp; pr < C * C; pr += nwarps) {
-        const int r = pr / C, i = pr % C;
-        float a = 0.f, pp = 0.f;
-        if (i <= r) {
-            for (int j = lane; j < dv; j += 32) {
-                const float u = U[(size_t)i * dv + j];
-                pp += dOs[(size_t)r * dv + j] * u;
-                a -= dR[(size_t)r * dv + j] * u;
-            }
-            a = warp_sum(a);
-            pp = warp_sum(pp);
+    // 5. dP = lower(dO U^T), dA = strictly-lower(-dR U^T).  Where U^T (rows padded to C + 1)
+    //    fits the free tile buffers: one thread per (r, i) pair with no cross-lane reduction
+    //    (a warp's lanes read consecutive i of U^T; dO and dR rows are broadcasts); otherwise
+    //    one warp per pair.
+    if ((size_t)dv * (C + 1) <= (size_t)2 * dk * kLd) {
+        float* Ut = St;
+        for (int idx = tid; idx < C * dv; idx += NT) {
+            const int i = idx / dv, j = idx % dv;
+            Ut[(size_t)j * (C + 1) + i] = U[idx];
         }
-        if (lane == 0) {
+        __syncthreads();
+        for (int pr = tid; pr < C * C; pr += NT) {
+            const int r = pr / C, i = pr % C;
+            float a = 0.f, pp = 0.f;
+            if (i <= r) {
+                for (int j = 0; j < dv; ++j) {
+                    const float u = Ut[(size_t)j * (C + 1) + i];
+                    pp += dOs[(size_t)r * dv + j] * u;
+                    a -= dR[(size_t)r * dv + j] * u;
+                }
+            }
             dA[pr] = (i < r) ? a : 0.f;
             dP[pr] = pp;
+        }
+    } else {
+        for (int pr = warp; pr < C * C; pr += nwarps) {
+            const int r = pr / C, i = pr % C;
+            float a = 0.f, pp = 0.f;
+            if (i <= r) {
+                for (int j = lane; j < dv; j += 32) {
+                    const float u = U[(size_t)i * dv + j];
+                    pp += dOs[(size_t)r * dv + j] * u;
+                    a -= dR[(size_t)r * dv + j] * u;
+                }
+                a = warp_sum(a);
+                pp = warp_sum(pp);
+            }
+            if (lane == 0) {
+                dA[pr] = (i < r) ? a : 0.f;
+                dP[pr] = pp;
+            }
         }
     }
     // 6. dO S^T, dR S^T, U dS'^T (thread: column cc, rows r0 + rstep * m) and rowsum(S (.) dS')
