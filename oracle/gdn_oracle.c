@@ -20,8 +20,7 @@
  *       S_t = X + k~_t (v~_t - X^T k~_t)^T
  *   which is the same matrix (expand (I - k~ k~^T) X + k~ v~^T).
  *
- *   Readings where the pages leave a step open (each one is listed in the
- *   design notes of the repository):
+ *   Readings where the pages leave a step open:
  *     - q and k arrive raw and are L2-normalised per token and head,
  *       x / sqrt(sum x^2 + eps), before k is scaled by sqrt(beta); no 1/sqrt(d)
  *       query scale is applied (none is mentioned).
