@@ -56,8 +56,6 @@ struct Problem {
     void* inter;            // per-chunk intermediates written by the intra role
     float* S_chunks;        // backward recompute: state at every chunk start,
                             // [B,H,NC,dk,dv]; null in the forward
-    int prefetch_ahead;     // intra role: CTAs per wave (SMs x resident CTAs); each CTA warms
-                            // L2 with the inputs of the CTA this far ahead in launch order
     // GDN2 (non-tied erase / write, float32 path only): eta [B,T,H] and b [B,T,H,dk]; the
     // erase vector is j' = eta k^ (.) b after the token-wise transform gdn2_mode
     // (0 none, 1 clip D to min(D, 1/rho), 2 shrink j' toward KDA); null eta: not GDN2.

@@ -366,32 +366,6 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     __half* fb_q = reinterpret_cast<__half*>(blk + kOffN);                // q^ fp16 [C][D]
     __half* fb_e = fb_q + C * D;                                          // GDN2 erase fp16 [C][D]
     cp_async_wait_all();     // this thread's own staged beta and v
-    // The CTAs of one wave load together and then compute with HBM idle.  Now that this
-    // CTA's inputs have arrived, start the next wave's: the CTA prefetch_ahead places
-    // later in launch order (x = chunk fastest) finds its rows in L2.
-    {
-        const long nxt = (long)blockIdx.y * gridDim.x + blockIdx.x + p.prefetch_ahead;
-        if (p.prefetch_ahead > 0 && nxt < (long)gridDim.x * gridDim.y) {
-            const int c2 = cb + (int)(nxt % gridDim.x), bh2 = (int)(nxt / gridDim.x);
-            const int r2 = tid >> 2, part = tid & 3;        // 4 threads per row
-            const int s2 = c2 * C + r2;
-            if (s2 < p.L) {
-                const RowRef rp = row_ref(p, bh2 / p.H, bh2 % p.H, s2);
-                const size_t kr2 = p.dp ? rp.tok * p.nh + rp.m : rp.tok;
-                // 128-byte lines: q, k, v rows 2 each (bf16), alpha / beta / beta_v rows 4 each
-                if (part < 2) {
-                    if (rp.has_q) prefetch_l2(q + rp.tok * D + 64 * part);
-                    prefetch_l2(k + kr2 * D + 64 * part);
-                    prefetch_l2(v + kr2 * D + 64 * part);
-                }
-                if (!a_scalar) prefetch_l2(p.alpha + rp.tok * D + 32 * part);
-                if (!b_scalar) {  // beta, or GDN2's gate b (p.beta is null there)
-                    prefetch_l2((kG2 ? p.gdn2_b : p.beta) + rp.tok * D + 32 * part);
-                    if (kPlus) prefetch_l2(p.beta_v + rp.tok * D + 32 * part);
-                }
-            }
-        }
-    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = o0 + 4 * j;
@@ -462,9 +436,13 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             QG[e] = qh * ex;
             KIG[e] = kt * exi;
             VT[e] = fv[e] * sv[e];
-            // fallback chunks: e^{-g} may overflow while e^{g_last} underflows, so take the
-            // ratio in one exponent there (it is <= 1)
-            KP[e] = fallback ? kt * __expf(glast[ch] - g[e]) : kt * exi * fK[ch];
+            KP[e] = KIG[e] * fK[ch];
+        }
+        if (fallback) {          // CTA-uniform: keeps the extra exponent off the common path
+            // e^{-g} may overflow while e^{g_last} underflows there, so take the ratio in one
+            // exponent (it is <= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) KP[e] = KT[e] * __expf(glast[8 * o + e] - g[e]);
         }
         const uint32_t off = off_kmajor(r, 8 * o, 2048, 128);
         st16(sm + kR0, off, f_to_h8(KG));
@@ -1079,21 +1057,10 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
                : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
     cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
     cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
-    Problem pi = p;
-    int dev = 0;
-    {
-        int sms = 0, per_sm = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, intra, tc::NT, tc::kIntraSmem) == cudaSuccess)
-            pi.prefetch_ahead = sms * per_sm;
-        else
-            pi.prefetch_ahead = 0;
-    }
     const dim3 g2(tc::J, p.B * p.H);
     const int P = tc_segments(p);
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream
-        intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, 0);
+        intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(p, 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
@@ -1111,7 +1078,7 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     for (int sg = 0; sg < P && e == cudaSuccess; ++sg) {
         int cb, ce;
         seg_range(p.NC, P, sg, cb, ce);
-        intra<<<dim3(ce - cb, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(pi, cb);
+        intra<<<dim3(ce - cb, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(p, cb);
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.ready[sg], 0);

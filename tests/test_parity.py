@@ -242,3 +242,14 @@ def test_tensor_core_segmented_call_uneven_ranges():
     cfg = GdnConfig("tcseg", B=1, H=2, T=64 * 97 + 13, dk=128, dv=128, chunk=64, s0_std=0.05, seed=6100)
     x = make_inputs(cfg)
     check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
+
+
+def test_tensor_core_large_offsets_sampled_heads():
+    """B5 H16 T32768: the workspace (40,960 chunk blocks, 4.7 GB) passes 2^32 bytes, so every
+    block offset must be 64-bit.  Sampled heads include the last one, whose blocks sit at the
+    top of the workspace."""
+    base = CONFIGS["fg2_prefill_32k"]
+    cfg = GdnConfig("large", B=5, H=16, T=base.T, dk=128, dv=128, chunk=64, s0_std=0.01, seed=6200)
+    x = make_inputs(cfg)
+    pairs = [(0, 0), (3, 9), (4, 15)]
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x, pairs=pairs), pairs=pairs)
