@@ -88,6 +88,10 @@ constexpr uint32_t kTmemCols = 256;
 // swizzled fp32 64x64: element (r, i)
 __device__ __forceinline__ int sw64(int r, int i) { return r * 64 + ((((i >> 2) ^ (r & 15))) << 2) + (i & 3); }
 
+// sqrt(x) for x >= 0 as x * rsqrt(x): a few ulp in fp32, far below the fp16 rounding of the
+// operands it scales, and shorter than the IEEE-rounded square root (x = 0 gives 0).
+__device__ __forceinline__ float sqrt_op(float x) { return x > 0.f ? x * rsqrtf(x) : 0.f; }
+
 __device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 __device__ __forceinline__ float4 ldg16f(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
 
@@ -174,6 +178,9 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     // into a staging area over R3..R6 (free until the solve), v straight into its final
     // place in R2 (converted in place later).  Everything is issued before any arithmetic.
     float* bstage = reinterpret_cast<float*>(sm + kR3);
+    // half h of octet o of row rr in the staging area: 16-byte units XOR-swizzled by the row,
+    // so eight consecutive rows reading the same unit hit eight different bank groups
+    auto bst = [bstage](int rr_, int o_, int h_) { return bstage + (rr_ * 32 + ((2 * o_ + h_) ^ (rr_ & 7))) * 4; };
     // Without beta^v, raw q and k also go to shared memory, into the R0 slots this thread
     // later overwrites with its own QG and KG octets; they are the first commit group, so
     // the norms wait for them alone.  (Holding them in registers through the norm and
@@ -202,9 +209,8 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
             const int o = o0 + 4 * j;
             if (!b_scalar) {      // beta, or GDN2's gate b (always channel-wise)
                 const float* bsrc = kG2 ? p.gdn2_b : p.beta;
-                float* dst = bstage + (r * 16 + (o ^ (r & 7))) * 8;
-                cp_async16(dst, bsrc + rr.tok * D + 8 * o);
-                cp_async16(dst + 4, bsrc + rr.tok * D + 8 * o + 4);
+                cp_async16(bst(r, o, 0), bsrc + rr.tok * D + 8 * o);
+                cp_async16(bst(r, o, 1), bsrc + rr.tok * D + 8 * o + 4);
             }
             cp_async16(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128), v + krow * D + 8 * o);
             if (kPlus && !b_scalar) {
@@ -276,14 +282,15 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int o = o0 + 4 * j;
-                const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+                const float* blo = bst(r, o, 0);
+                const float* bhi = bst(r, o, 1);
                 float fk[8];
                 bf8_to_f(kp[j], fk);
                 const float a8[8] = {al0[j].x, al0[j].y, al0[j].z, al0[j].w, al1[j].x, al1[j].y, al1[j].z, al1[j].w};
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float kh = fk[e] * ik;
-                    const float jp = g2_eta * kh * bsrc[e];
+                    const float jp = g2_eta * kh * (e < 4 ? blo[e] : bhi[e - 4]);
                     cd += jp * kh;
                     nj += jp * jp;
                     am = fmaxf(am, a_scalar ? as_ : a8[e]);
@@ -373,22 +380,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) g[e] = la[j][e] + scr[warp * D + 8 * o + e];
         if (kG2) {                // no beta: k~ = k^; the gate b feeds the erase vector
-            const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
+            const float* blo = bst(r, o, 0);
+            const float* bhi = bst(r, o, 1);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 sb[e] = valid ? 1.f : 0.f;
-                gb[e] = valid ? bsrc[e] : 0.f;
+                gb[e] = valid ? (e < 4 ? blo[e] : bhi[e - 4]) : 0.f;
             }
         } else if (b_scalar || !valid) {
             const float s = valid ? sqrtf(b_s) : 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) sb[e] = s;
         } else {
-            const float* bsrc = bstage + (r * 16 + (o ^ (r & 7))) * 8;
-            const float4 b0 = *reinterpret_cast<const float4*>(bsrc);
-            const float4 b1 = *reinterpret_cast<const float4*>(bsrc + 4);
-            sb[0] = sqrtf(b0.x); sb[1] = sqrtf(b0.y); sb[2] = sqrtf(b0.z); sb[3] = sqrtf(b0.w);
-            sb[4] = sqrtf(b1.x); sb[5] = sqrtf(b1.y); sb[6] = sqrtf(b1.z); sb[7] = sqrtf(b1.w);
+            const float4 b0 = *reinterpret_cast<const float4*>(bst(r, o, 0));
+            const float4 b1 = *reinterpret_cast<const float4*>(bst(r, o, 1));
+            sb[0] = sqrt_op(b0.x); sb[1] = sqrt_op(b0.y); sb[2] = sqrt_op(b0.z); sb[3] = sqrt_op(b0.w);
+            sb[4] = sqrt_op(b1.x); sb[5] = sqrt_op(b1.y); sb[6] = sqrt_op(b1.z); sb[7] = sqrt_op(b1.w);
         }
         if (kG2) {
 #pragma unroll
@@ -403,8 +410,8 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
         } else {
             const float4 b0 = *reinterpret_cast<const float4*>(sm + kR0 + off_kmajor(r, 8 * o, 2048, 128));
             const float4 b1 = *reinterpret_cast<const float4*>(sm + kR0 + off_kmajor(64 + r, 8 * o, 2048, 128));
-            sv[0] = sqrtf(b0.x); sv[1] = sqrtf(b0.y); sv[2] = sqrtf(b0.z); sv[3] = sqrtf(b0.w);
-            sv[4] = sqrtf(b1.x); sv[5] = sqrtf(b1.y); sv[6] = sqrtf(b1.z); sv[7] = sqrtf(b1.w);
+            sv[0] = sqrt_op(b0.x); sv[1] = sqrt_op(b0.y); sv[2] = sqrt_op(b0.z); sv[3] = sqrt_op(b0.w);
+            sv[4] = sqrt_op(b1.x); sv[5] = sqrt_op(b1.y); sv[6] = sqrt_op(b1.z); sv[7] = sqrt_op(b1.w);
         }
         const uint4 vp = valid ? *reinterpret_cast<const uint4*>(sm + kR2 + off_kmajor(r, 8 * o, 2048, 128))
                                : make_uint4(0, 0, 0, 0);
@@ -466,9 +473,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     const uint32_t t0 = *tslot;
     bool ok = true;
     uint32_t phase = 0;      // parity of the next completion of `bar`
-    // identity operand (B layout: n = r, k = i); its area held staged beta until now
+    // identity operand (B layout: n = r, k = i); its area held staged beta until now.
+    // Eight consecutive lanes take eight consecutive rows: one 128-byte line per store phase.
     for (int idx = tid; idx < 512; idx += NT) {
-        const int ri = idx >> 3, j = idx & 7;
+        const int ri = idx & 63, j = idx >> 6;
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = (8 * j + e == ri) ? 1.f : 0.f;
@@ -625,13 +633,15 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     }
     __syncthreads();
     for (int idx = tid; idx < 512; idx += NT) {   // T -> fp16 B operand (n = r, k = i)
-        const int rw = idx >> 3, j = idx & 7;
-        float f[8];
+        // eight consecutive lanes take eight consecutive rows: the swizzled float4 reads and
+        // the 16-byte stores both fall in distinct bank groups
+        const int rw = idx & 63, j = idx >> 6;
+        const float4 ta = *reinterpret_cast<const float4*>(T32 + sw64(rw, 8 * j));
+        const float4 tb = *reinterpret_cast<const float4*>(T32 + sw64(rw, 8 * j + 4));
+        float f[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int i = 8 * j + e;
-            f[e] = (i <= rw) ? T32[sw64(rw, i)] : 0.f;
-        }
+        for (int e = 0; e < 8; ++e)
+            if (8 * j + e > rw) f[e] = 0.f;
         st16(sm + kR3, off_kmajor(rw, 8 * j, 1024, 128), f_to_h8(f));
     }
     fence_async_smem();
@@ -777,65 +787,87 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 }
 
 // ============================================================================ scan
-// One CTA per (head, 32-column slice).  Per chunk c, with S_c in fp32 registers (row i
-// per thread) and its fp16 copy in Sop[c % 3]:
+// One CTA per (head, W consecutive 32-column slices).  Per chunk c, with S_c in fp32
+// registers (row i per thread, 32 columns per warp) and its fp16 copy in Sop[c % 3]:
 //   MMA_S: D_S = N_c S_c          -> S_{c+1} = Diag(gC) S_c + D_S + b_c   (the serial chain)
 //   MMA_O: D_O[c & 1] = Qe_c S_c  -> O_c = D_O + PU'_c                     (off the chain)
 // MMA_O(c) is issued right after MMA_S(c+1), so it runs in the tensor pipe while the state
 // epilogue of chunk c+1 works instead of sitting in front of the next chain MMA; the fp16
 // state therefore keeps three buffers.
-// Roles: warps 0-3 carry the state (one d_k row per thread), warps 4-7 form the outputs
-// (the M = 64 accumulator puts row r in lane (r%16) + 32*(r/16)), warp 8 streams the
-// per-chunk blocks with bulk copies into two rings ({N, b slice, gC} x 3 and
-// {Qe, PU' slice} x 4), and one thread of warp 9 issues every MMA.  All hand-offs are
-// mbarriers with bounded waits.
-constexpr int kScanThreads = 320;
-constexpr int kNB = 3, kQP = 4;
-constexpr uint32_t kNBBytes = 32768 + 8192 + 512;
-constexpr uint32_t kNBStride = 41472;
-constexpr uint32_t kQPBytes = 16384 + 4096;
-constexpr uint32_t kQPStride = 20480;
-constexpr uint32_t kSN = 0, kSB = 32768, kSG = 40960;      // within an NB stage
-constexpr uint32_t kSQe = 0, kSPU = 16384;                 // within a QP stage
-constexpr uint32_t kRingNB = 0;
-constexpr uint32_t kRingQP = kRingNB + kNB * kNBStride;    // 124416
-constexpr uint32_t kSop = kRingQP + kQP * kQPStride;       // 206336: 3 x 8 KB, S fp16 (k = i, n = j) MN-major SBO 2048 LBO 128
-constexpr uint32_t kSBar = kSop + 3 * 8192;                // 230912: mbarriers
-constexpr uint32_t kSTmem = kSBar + 256;
-constexpr uint32_t kScanSmem = kSTmem + 64;                // 231232
+// Roles: warps 0 .. 4W-1 carry the state (warp w: TMEM lane quarter w % 4, slice w / 4),
+// warps 4W .. 4W+3 form the outputs of all W slices in turn (the M = 64 accumulator puts
+// row r in lane (r%16) + 32*(r/16)), warp 4W+4 streams the per-chunk blocks with bulk copies
+// into two rings ({N, b slices, gC} and {Qe, PU' slices}), and one thread of warp 4W+5
+// issues every MMA.  All hand-offs are mbarriers with bounded waits.  (Four output warps
+// rather than 4W keep at most four warps on each scheduler, so the register budget per
+// thread stays at 128.  One producer warp per ring, an L2 prefetch of the blocks a few
+// chunks ahead, and reading every slice's D_O before freeing it were each measured slower.)
+// The chain MMA costs about the same for N = 32 and N = 64 (its latency is the tensor pipe's,
+// not the columns'), so W = 2 carries a head's state on half as many SMs.  Its step is slower
+// (twice the state warps per scheduler, a shallower ring), so launch_tc takes W = 2 only when
+// the W = 1 grid would need more than one wave of SMs.
+template <int W>
+struct ScanCfg {
+    static constexpr int kThreads = 32 * (4 * W + 6);
+    static constexpr int kNB = W == 1 ? 3 : 2;             // ring depths (shared memory bound)
+    static constexpr int kQP = W == 1 ? 4 : 3;
+    static constexpr uint32_t kNBBytes = 32768 + 8192 * W + 512;
+    static constexpr uint32_t kNBStride = kNBBytes;        // a 128-byte multiple
+    static constexpr uint32_t kSN = 0, kSB = 32768, kSG = 32768 + 8192 * W;   // within an NB stage
+    static constexpr uint32_t kQPBytes = 16384 + 4096 * W;
+    static constexpr uint32_t kQPStride = kQPBytes;
+    static constexpr uint32_t kSQe = 0, kSPU = 16384;                        // within a QP stage
+    static constexpr uint32_t kRingNB = 0;
+    static constexpr uint32_t kRingQP = kRingNB + kNB * kNBStride;
+    static constexpr uint32_t kSopBytes = 8192 * W;        // S fp16 (k = i, n = j) MN-major SBO 2048 LBO 128
+    static constexpr uint32_t kSop = kRingQP + kQP * kQPStride;
+    static constexpr uint32_t kSBar = kSop + 3 * kSopBytes;
+    static constexpr uint32_t kSTmem = kSBar + 256;
+    static constexpr uint32_t kSmem = kSTmem + 64;
+    static constexpr uint32_t kTmemCols = W == 1 ? 128 : 256;   // D_S (32W) + 2 x D_O (32W)
+};
+static_assert(ScanCfg<1>::kSmem == 231232 && ScanCfg<2>::kSmem <= 232448 - 1024, "scan shared memory");
+static_assert(ScanCfg<1>::kNBBytes % 128 == 0 && ScanCfg<2>::kNBBytes % 128 == 0 &&
+              ScanCfg<2>::kSop % 1024 == 0, "stage alignment");
+static_assert(2 * ScanCfg<1>::kNB + 2 * ScanCfg<1>::kQP + 6 <= 32 &&
+              2 * ScanCfg<2>::kNB + 2 * ScanCfg<2>::kQP + 6 <= 32, "mbarrier area");
 
 // This launch covers chunks cb .. ce-1, starting from S_in (null: zero) and leaving the
 // state in S_out (may be null); ring stages and barrier phases count from cb.
-__global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int cb, int ce,
-                                                                  const float* S_in, float* S_out) {
+template <int W>
+__global__ void __launch_bounds__(ScanCfg<W>::kThreads, 1) scan_tc_kernel(Problem p, int cb, int ce,
+                                                                         const float* S_in, float* S_out) {
+    using Cfg = ScanCfg<W>;
+    constexpr int kNB = Cfg::kNB, kQP = Cfg::kQP;
+    constexpr int NSW = NS * W;                            // columns of this CTA
     extern __shared__ __align__(1024) uint8_t sm[];
-    const int slice = blockIdx.x;
+    const int slice0 = blockIdx.x * W;                     // first 32-column slice of this CTA
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t* fullNB = reinterpret_cast<uint64_t*>(sm + kSBar);
+    uint64_t* fullNB = reinterpret_cast<uint64_t*>(sm + Cfg::kSBar);
     uint64_t* emptyNB = fullNB + kNB;
     uint64_t* fullQP = emptyNB + kNB;
     uint64_t* emptyQP = fullQP + kQP;
     uint64_t* bar_s = emptyQP + kQP;       // MMA_S done
     uint64_t* bar_o = bar_s + 1;           // [2] MMA_O done, per D_O buffer
-    uint64_t* s_ready = bar_o + 2;         // S_c written to Sop (4 warp arrivals)
+    uint64_t* s_ready = bar_o + 2;         // S_c written to Sop (4W warp arrivals)
     uint64_t* o_free = s_ready + 1;        // [2] D_O buffer read (4 warp arrivals)
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kSTmem);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + Cfg::kSTmem);
     const uint8_t* blocks = static_cast<const uint8_t*>(p.inter) + (size_t)bh * p.NC * kBlockBytes;
     const int nloc = ce - cb;              // chunks of this launch; loop indices below are local
 
     if (warp == 0) {
-        tmem_alloc(tslot, 128);
+        tmem_alloc(tslot, Cfg::kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < kNB; ++i) { mbar_init(&fullNB[i], 1); mbar_init(&emptyNB[i], 4); }
+        for (int i = 0; i < kNB; ++i) { mbar_init(&fullNB[i], 1); mbar_init(&emptyNB[i], 4 * W); }
         for (int i = 0; i < kQP; ++i) { mbar_init(&fullQP[i], 1); mbar_init(&emptyQP[i], 4); }
         mbar_init(bar_s, 1);
         mbar_init(&bar_o[0], 1);
         mbar_init(&bar_o[1], 1);
-        mbar_init(s_ready, 4);
+        mbar_init(s_ready, 4 * W);
         mbar_init(&o_free[0], 4);
         mbar_init(&o_free[1], 4);
         fence_mbar_init();
@@ -844,44 +876,44 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
     __syncthreads();
     tc_fence_after();
     const uint32_t t0 = *tslot;
-    const uint32_t tS = t0, tO = t0 + 32;                  // D_S (32 columns); D_O[0], D_O[1]
+    const uint32_t tS = t0, tO = t0 + NSW;                 // D_S (NSW columns); D_O[0], D_O[1]
     bool ok = true;
 
-    if (warp == 8) {
+    if (warp == 4 * W + 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             for (int ch = 0; ch < nloc && ok; ++ch) {
                 const uint8_t* src = blocks + (size_t)(cb + ch) * kBlockBytes;
                 const int s3 = ch % kNB, s4 = ch % kQP;
                 if (ch >= kNB && !mbar_wait(&emptyNB[s3], ((ch / kNB) - 1) & 1)) { ok = false; break; }
-                uint8_t* d3 = sm + kRingNB + s3 * kNBStride;
-                mbar_arrive_expect_tx(&fullNB[s3], kNBBytes);
-                bulk_g2s(d3 + kSN, src + kOffN, 32768, &fullNB[s3]);
-                bulk_g2s(d3 + kSB, src + kOffB + (size_t)slice * D * NS * 2, 8192, &fullNB[s3]);
-                bulk_g2s(d3 + kSG, src + kOffGC, 512, &fullNB[s3]);
+                uint8_t* d3 = sm + Cfg::kRingNB + s3 * Cfg::kNBStride;
+                mbar_arrive_expect_tx(&fullNB[s3], Cfg::kNBBytes);
+                bulk_g2s(d3 + Cfg::kSN, src + kOffN, 32768, &fullNB[s3]);
+                bulk_g2s(d3 + Cfg::kSB, src + kOffB + (size_t)slice0 * D * NS * 2, 8192 * W, &fullNB[s3]);
+                bulk_g2s(d3 + Cfg::kSG, src + kOffGC, 512, &fullNB[s3]);
                 if (ch >= kQP && !mbar_wait(&emptyQP[s4], ((ch / kQP) - 1) & 1)) { ok = false; break; }
-                uint8_t* d4 = sm + kRingQP + s4 * kQPStride;
-                mbar_arrive_expect_tx(&fullQP[s4], kQPBytes);
-                bulk_g2s(d4 + kSQe, src + kOffQe, 16384, &fullQP[s4]);
-                bulk_g2s(d4 + kSPU, src + kOffPU + (size_t)slice * C * NS * 2, 4096, &fullQP[s4]);
+                uint8_t* d4 = sm + Cfg::kRingQP + s4 * Cfg::kQPStride;
+                mbar_arrive_expect_tx(&fullQP[s4], Cfg::kQPBytes);
+                bulk_g2s(d4 + Cfg::kSQe, src + kOffQe, 16384, &fullQP[s4]);
+                bulk_g2s(d4 + Cfg::kSPU, src + kOffPU + (size_t)slice0 * C * NS * 2, 4096 * W, &fullQP[s4]);
             }
             if (!ok) record_timeout(p.status);
         }
-    } else if (warp == 9) {
+    } else if (warp == 4 * W + 5) {
         // ------------------------------------------------------------ MMA issuer (one thread)
         if (lane == 0) {
-            const uint32_t idS = idesc_f16(128, NS, false, true);
-            const uint32_t idO = idesc_f16(64, NS, true, true);
+            const uint32_t idS = idesc_f16(128, NSW, false, true);
+            const uint32_t idO = idesc_f16(64, NSW, true, true);
             // MMA_O of chunk cc (reads Sop[cc % 3] and the QP stage of cc)
             auto issue_o = [&](int cc) -> bool {
                 const int s4 = cc % kQP;
                 if (cc >= 2 && !mbar_wait(&o_free[cc & 1], ((cc >> 1) - 1) & 1)) return false;
                 if (!mbar_wait(&fullQP[s4], (cc / kQP) & 1)) return false;
                 tc_fence_after();
-                const uint64_t a0 = sdesc(smem_u32(sm + kRingQP + s4 * kQPStride + kSQe), 128, 2048);
-                const uint64_t b0 = sdesc(smem_u32(sm + kSop + (cc % 3) * 8192), 128, 2048);
+                const uint64_t a0 = sdesc(smem_u32(sm + Cfg::kRingQP + s4 * Cfg::kQPStride + Cfg::kSQe), 128, 2048);
+                const uint64_t b0 = sdesc(smem_u32(sm + Cfg::kSop + (cc % 3) * Cfg::kSopBytes), 128, 2048);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) mma_f16(tO + 32 * (cc & 1), a0 + 16 * kk, b0 + 16 * kk, idO, kk > 0);
+                for (int kk = 0; kk < D / 16; ++kk) mma_f16(tO + NSW * (cc & 1), a0 + 16 * kk, b0 + 16 * kk, idO, kk > 0);
                 mma_commit(&bar_o[cc & 1]);
                 return true;
             };
@@ -890,8 +922,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
                 if (!mbar_wait(s_ready, ch & 1) || !mbar_wait(&fullNB[s3], (ch / kNB) & 1)) { ok = false; break; }
                 tc_fence_after();
                 {
-                    const uint64_t a0 = sdesc(smem_u32(sm + kRingNB + s3 * kNBStride + kSN), 128, 2048);
-                    const uint64_t b0 = sdesc(smem_u32(sm + kSop + (ch % 3) * 8192), 128, 2048);
+                    const uint64_t a0 = sdesc(smem_u32(sm + Cfg::kRingNB + s3 * Cfg::kNBStride + Cfg::kSN), 128, 2048);
+                    const uint64_t b0 = sdesc(smem_u32(sm + Cfg::kSop + (ch % 3) * Cfg::kSopBytes), 128, 2048);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) mma_f16(tS, a0 + 16 * kk, b0 + 16 * kk, idS, kk > 0);
                     mma_commit(bar_s);
@@ -901,24 +933,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
             if (ok && nloc > 0) ok = issue_o(nloc - 1);
             if (!ok) record_timeout(p.status);
         }
-    } else if (warp < 4) {
+    } else if (warp < 4 * W) {
         // ------------------------------------------------------------ state chain
-        const int row = tid;                                   // d_k row of S (TMEM lane)
-        const int j0 = slice * NS;
-        const uint32_t lanebase = (uint32_t)(32 * warp) << 16;
+        const int q = warp & 3, sl = warp >> 2;                // TMEM lane quarter, slice within the CTA
+        const int row = 32 * q + lane;                         // d_k row of S (TMEM lane)
+        const int j0 = (slice0 + sl) * NS;                     // first state column of this warp
+        const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         float S[NS];
 #pragma unroll
         for (int j = 0; j < NS; ++j) S[j] = S_in ? S_in[((size_t)bh * D + row) * D + j0 + j] : 0.f;
 #pragma unroll
-        for (int j = 0; j < NS; j += 8) st16(sm + kSop, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
+        for (int j = 0; j < NS; j += 8) st16(sm + Cfg::kSop, off_mnmajor(NS * sl + j, row, 2048, 128), f_to_h8(S + j));
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_ready);
         for (int ch = 0; ch < nloc && ok; ++ch) {
             const int s3 = ch % kNB;
-            const uint8_t* nb = sm + kRingNB + s3 * kNBStride;
+            const uint8_t* nb = sm + Cfg::kRingNB + s3 * Cfg::kNBStride;
             if (!__all_sync(0xffffffffu, mbar_wait(&fullNB[s3], (ch / kNB) & 1))) { ok = false; break; }
-            const __half* bsm = reinterpret_cast<const __half*>(nb + kSB);
+            const __half* bsm = reinterpret_cast<const __half*>(nb + Cfg::kSB) + sl * (D * NS);
             float bv[NS];
 #pragma unroll
             for (int g8 = 0; g8 < NS; g8 += 8) {
@@ -931,21 +964,21 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
                     bv[g8 + 2 * e + 1] = f.y;
                 }
             }
-            const float gc = reinterpret_cast<const float*>(nb + kSG)[row];
+            const float gc = reinterpret_cast<const float*>(nb + Cfg::kSG)[row];
             if (!__all_sync(0xffffffffu, mbar_wait(bar_s, ch & 1))) { ok = false; break; }
             tc_fence_after();
             float d[NS];
-            tmem_ld32(t0 + lanebase + (tS - t0), d);
+            tmem_ld32(tS + lanebase + NS * sl, d);
 #pragma unroll
             for (int j = 0; j < NS; ++j) S[j] = fmaf(gc, S[j], d[j] + bv[j]);
-            uint8_t* snext = sm + kSop + ((ch + 1) % 3) * 8192;
+            uint8_t* snext = sm + Cfg::kSop + ((ch + 1) % 3) * Cfg::kSopBytes;
 #pragma unroll
-            for (int j = 0; j < NS; j += 8) st16(snext, off_mnmajor(j, row, 2048, 128), f_to_h8(S + j));
+            for (int j = 0; j < NS; j += 8) st16(snext, off_mnmajor(NS * sl + j, row, 2048, 128), f_to_h8(S + j));
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(s_ready);                          // S_{ch+1} is in Sop[(ch+1) % 3]
+                mbar_arrive(s_ready);                          // this warp's part of S_{ch+1} is in Sop
                 mbar_arrive(&emptyNB[s3]);
             }
         }
@@ -957,11 +990,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
             for (int j = 0; j < NS; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
     } else {
-        // ------------------------------------------------------------ outputs (warps 4-7)
-        const int wq = warp - 4;                               // TMEM lane quarter
-        const int j0 = slice * NS;
-        const uint32_t lanebase = (uint32_t)(32 * wq) << 16;
-        const int rw = 16 * wq + lane;                         // output row (valid for lane < 16)
+        // ------------------------------------------------------------ outputs (warps 4W .. 4W+3)
+        const int q = warp - 4 * W;                            // TMEM lane quarter
+        const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+        const int rw = 16 * q + lane;                          // output row (valid for lane < 16)
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         for (int ch = 0; ch < nloc && ok; ++ch) {
             const int s4 = ch % kQP;
@@ -971,30 +1003,33 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
                 break;
             }
             tc_fence_after();
-            float d[NS];
-            tmem_ld32(t0 + lanebase + (tO - t0) + 32 * (ch & 1), d);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&o_free[ch & 1]);
-            if (lane < 16) {
-                const int s = (cb + ch) * C + rw;
-                if (s < p.L) {
-                    const RowRef ro = row_ref(p, b, h, s);
-                    if (ro.has_q) {
-                        const __half* pu = reinterpret_cast<const __half*>(sm + kRingQP + s4 * kQPStride + kSPU);
-                        uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + j0);
+            const int s = (cb + ch) * C + rw;
+            RowRef ro{};
+            const bool write = lane < 16 && s < p.L && (ro = row_ref(p, b, h, s)).has_q;
+#pragma unroll 1
+            for (int sl = 0; sl < W; ++sl) {
+                float d[NS];
+                tmem_ld32(tO + lanebase + NSW * (ch & 1) + NS * sl, d);
+                if (sl == W - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&o_free[ch & 1]);
+                }
+                if (write) {
+                    const __half* pu = reinterpret_cast<const __half*>(sm + Cfg::kRingQP + s4 * Cfg::kQPStride + Cfg::kSPU) +
+                                       sl * (C * NS);
+                    uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + (slice0 + sl) * NS);
 #pragma unroll
-                        for (int g8 = 0; g8 < NS; g8 += 8) {
-                            const uint4 pv = *reinterpret_cast<const uint4*>(pu + sw_half(rw, g8));
-                            const __half2* ph = reinterpret_cast<const __half2*>(&pv);
-                            __nv_bfloat162 o2[4];
+                    for (int g8 = 0; g8 < NS; g8 += 8) {
+                        const uint4 pv = *reinterpret_cast<const uint4*>(pu + sw_half(rw, g8));
+                        const __half2* ph = reinterpret_cast<const __half2*>(&pv);
+                        __nv_bfloat162 o2[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 pf = __half22float2(ph[e]);
-                                o2[e] = __floats2bfloat162_rn(pf.x + d[g8 + 2 * e], pf.y + d[g8 + 2 * e + 1]);
-                            }
-                            dst[g8 / 8] = *reinterpret_cast<uint4*>(o2);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 pf = __half22float2(ph[e]);
+                            o2[e] = __floats2bfloat162_rn(pf.x + d[g8 + 2 * e], pf.y + d[g8 + 2 * e + 1]);
                         }
+                        dst[g8 / 8] = *reinterpret_cast<uint4*>(o2);
                     }
                 }
             }
@@ -1005,7 +1040,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_tc_kernel(Problem p, int
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(t0, 128);
+    if (warp == 0) tmem_dealloc(t0, Cfg::kTmemCols);
 }
 
 }  // namespace tc
@@ -1056,14 +1091,22 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
                : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
     cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
-    cudaFuncSetAttribute(tc::scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kScanSmem);
-    const dim3 g2(tc::J, p.B * p.H);
+    // scan width: two slices per CTA when one slice per CTA would take more than one wave
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 0;
+    const bool w2 = (long)p.B * p.H * tc::J > (long)sms;
+    auto scan = w2 ? tc::scan_tc_kernel<2> : tc::scan_tc_kernel<1>;
+    const uint32_t scan_smem = w2 ? tc::ScanCfg<2>::kSmem : tc::ScanCfg<1>::kSmem;
+    const int scan_threads = w2 ? tc::ScanCfg<2>::kThreads : tc::ScanCfg<1>::kThreads;
+    cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    const dim3 g2(tc::J / (w2 ? 2 : 1), p.B * p.H);
     const int P = tc_segments(p);
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream
         intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(p, 0);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
+        scan<<<g2, scan_threads, scan_smem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
         return cudaGetLastError();
     };
     if (P == 1) return one_stream();
@@ -1083,7 +1126,7 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
         if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.ready[sg], 0);
         if (e != cudaSuccess) break;
-        tc::scan_tc_kernel<<<g2, tc::kScanThreads, tc::kScanSmem, ss.stream>>>(
+        scan<<<g2, scan_threads, scan_smem, ss.stream>>>(
             p, cb, ce, sg == 0 ? p.S0 : handoff, sg == P - 1 ? p.S_final : handoff);
         e = cudaGetLastError();
     }

@@ -253,3 +253,13 @@ def test_tensor_core_large_offsets_sampled_heads():
     x = make_inputs(cfg)
     pairs = [(0, 0), (3, 9), (4, 15)]
     check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x, pairs=pairs), pairs=pairs)
+
+
+@pytest.mark.parametrize("T,pairs", [(64 * 3 + 17, None), (64 * 70 + 5, [(0, 0), (5, 2), (9, 3)])])
+def test_tensor_core_wide_scan_grid(T, pairs):
+    """B10 H4: one 32-column slice per scan CTA would need 160 CTAs, more than one wave of
+    SMs, so the scan carries two slices per CTA.  Short (every head checked) and segmented
+    (sampled heads) calls, nonzero S0."""
+    cfg = GdnConfig("tcw2", B=10, H=4, T=T, dk=128, dv=128, chunk=64, s0_std=0.05, seed=6300 + T)
+    x = make_inputs(cfg)
+    check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x, pairs=pairs), pairs=pairs)
