@@ -153,9 +153,9 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def cpu_baseline(cfg, budget_s: float = 12.0):
+def cpu_baseline(cfg, target_s: float = 12.0):
     """Time the fp64 oracle (as it stands) on a bounded sample: whole heads of the
-    workload, as many as fit the budget, one head per thread."""
+    workload, as many as fit in about target_s seconds, one head per thread."""
     import oracle
     threads = oracle.max_threads()
     x = make_inputs(cfg, T=min(cfg.T, 2048), H=1, B=1)
@@ -166,9 +166,9 @@ def cpu_baseline(cfg, budget_s: float = 12.0):
         oracle.gdn_seq(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
                        alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar, nthreads=1)
     per_tok_head = (time.perf_counter() - t0) / x["q"].shape[1]
-    # heads run in parallel, one per thread; pick a sample of whole heads that fits the budget
+    # heads run in parallel, one per thread; pick a sample of whole heads that fits target_s
     nheads = max(1, min(cfg.B * cfg.H, threads))
-    T_s = int(max(256, min(cfg.T, budget_s / max(per_tok_head, 1e-9))))
+    T_s = int(max(256, min(cfg.T, target_s / max(per_tok_head, 1e-9))))
     H_s = min(cfg.H, nheads)
     x = make_inputs(cfg, T=T_s, H=H_s, B=1)
     t0 = time.perf_counter()
@@ -191,11 +191,11 @@ def run_reference(args, cfg):
         return
     vals, last = [], None
     # each step is a bounded sample, sized so that warm-up + timed steps end within minutes
-    budget = max(0.5, min(args.ref_budget, 150.0 / max(1, args.steps + args.warmup)))
+    per_step_s = max(0.5, min(args.ref_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(max(0, args.warmup)):
-        cpu_baseline(cfg, budget_s=budget)
+        cpu_baseline(cfg, target_s=per_step_s)
     for _ in range(args.steps):
-        last = cpu_baseline(cfg, budget_s=budget)
+        last = cpu_baseline(cfg, target_s=per_step_s)
         vals.append(last["value"])
     v = float(np.median(vals))
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
@@ -366,7 +366,7 @@ def main():
                          "recurrent step per sequence (B=256 by default); bwd: the chunked backward; "
                          "gdn2: GDN2 with the decay clip")
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--ref-budget", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up + timed steps (no clock soak, e2e or CPU baseline), for ncu")

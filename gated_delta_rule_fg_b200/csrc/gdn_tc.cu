@@ -799,8 +799,8 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
 // row r in lane (r%16) + 32*(r/16)), warp 4W+4 streams the per-chunk blocks with bulk copies
 // into two rings ({N, b slices, gC} and {Qe, PU' slices}), and one thread of warp 4W+5
 // issues every MMA.  All hand-offs are mbarriers with bounded waits.  (Four output warps
-// rather than 4W keep at most four warps on each scheduler, so the register budget per
-// thread stays at 128.  One producer warp per ring, an L2 prefetch of the blocks a few
+// rather than 4W keep at most four warps on each scheduler, so each thread may keep
+// up to 128 registers.  One producer warp per ring, an L2 prefetch of the blocks a few
 // chunks ahead, and reading every slice's D_O before freeing it were each measured slower.)
 // The chain MMA costs about the same for N = 32 and N = 64 (its latency is the tensor pipe's,
 // not the columns'), so W = 2 carries a head's state on half as many SMs.  Its step is slower

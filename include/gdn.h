@@ -70,7 +70,7 @@ extern "C" {
 typedef enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1,   /* NULL / misaligned pointer, negative size, dk != dv with channel-wise beta */
-    GDN_ERR_UNSUPPORTED = 2,   /* a size this build does not implement (see gdn_chunk_fwd) */
+    GDN_ERR_UNSUPPORTED = 2,   /* a size the library does not implement (see gdn_chunk_fwd) */
     GDN_ERR_CUDA = 3,          /* a CUDA launch or copy failed (cudaGetLastError is left set) */
     GDN_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out; outputs are not valid */
     GDN_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or smaller than required */
