@@ -25,7 +25,7 @@ constexpr int kR = NT / kG;      // row groups (16)
 template <typename Tin, int DK>
 __global__ void __launch_bounds__(NT) step_kernel(Problem p) {
     constexpr int RPT = DK / kR;             // rows per thread
-    __shared__ float s_qa[DK], s_ka[DK], s_kt[DK];
+    __shared__ float s_qa[DK], s_ka[DK], s_kt[DK], s_al[DK];
     __shared__ float s_red[3][NT / 32];
     __shared__ float s_pa[kR][kCols], s_pc[kR][kCols];
     __shared__ float s_u[kCols];
@@ -37,6 +37,19 @@ __global__ void __launch_bounds__(NT) step_kernel(Problem p) {
     const int dk = DK, dv = p.dv;
     const Tin* q = static_cast<const Tin*>(p.q) + (size_t)bh * dk;
     const Tin* k = static_cast<const Tin*>(p.k) + (size_t)bh * dk;
+
+    // the state slice first: its loads do not depend on the token prep, so they are in
+    // flight while the prep's loads and reductions run
+    const int rg = tid / kG, cg = tid % kG;
+    const int c = col0 + 4 * cg;
+    float4 s[RPT];
+    const size_t sbase = (size_t)bh * dk * dv;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int i = rg + kR * m;
+        s[m] = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)i * dv + c)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 
     // token prep: norms of q and k, and q^ . k~ (needs sqrt(beta^k) per channel)
     float xq = 0.f, xk = 0.f, a = 1.f, sb = 0.f;
@@ -67,20 +80,11 @@ __global__ void __launch_bounds__(NT) step_kernel(Problem p) {
         s_qa[tid] = xq * iq * a;
         s_ka[tid] = kt * a;
         s_kt[tid] = kt;
+        s_al[tid] = a;
     }
     __syncthreads();
 
     // one pass over the slice: X^T k~ and (alpha (.) q^)^T S per column
-    const int rg = tid / kG, cg = tid % kG;
-    const int c = col0 + 4 * cg;
-    float4 s[RPT];
-    const size_t sbase = (size_t)bh * dk * dv;
-#pragma unroll
-    for (int m = 0; m < RPT; ++m) {
-        const int i = rg + kR * m;
-        s[m] = p.S0 ? *reinterpret_cast<const float4*>(p.S0 + sbase + (size_t)i * dv + c)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     float pa[4] = {0.f, 0.f, 0.f, 0.f}, pc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(NT) step_kernel(Problem p) {
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
         const int i = rg + kR * m;
-        const float al = p.alpha_scalar ? p.alpha[bh] : p.alpha[(size_t)bh * dk + i];
+        const float al = s_al[i];
         const float kt = s_kt[i];
         float4 r;
         r.x = al * s[m].x + kt * u0;
