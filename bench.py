@@ -92,16 +92,47 @@ def load_traffic(kernel: str, workload: str, source_hash: str):
 TC_SOURCES = ("gdn_tc.cu", "gdn_sm100.cuh")     # the timed kernels' own code
 
 
+def code_only(text: str) -> str:
+    """C/CUDA source without its comments and trailing blanks: what the compiler sees as
+    code, so that an edit of a comment does not count as a change of the kernel."""
+    out, i, n, in_str = [], 0, len(text), None
+    while i < n:
+        c = text[i]
+        if in_str:
+            out.append(c)
+            if c == "\\" and i + 1 < n:
+                out.append(text[i + 1])
+                i += 1
+            elif c == in_str:
+                in_str = None
+        elif c in "\"'":
+            in_str = c
+            out.append(c)
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+            continue
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            continue
+        else:
+            out.append(c)
+        i += 1
+    lines = (l.rstrip() for l in "".join(out).splitlines())
+    return "\n".join(l for l in lines if l)
+
+
 def source_hash() -> str:
-    """Hash of the sources of the kernels bench.py times; traffic counters taken on other
-    sources are not reported."""
+    """Hash of the code (comments dropped) of the kernels bench.py times; traffic counters
+    taken on other code are not reported."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_fg_b200", "csrc")
     for n in TC_SOURCES:
-        with open(os.path.join(csrc, n), "rb") as f:
+        with open(os.path.join(csrc, n), encoding="utf-8") as f:
             h.update(n.encode())
-            h.update(f.read())
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -18,8 +18,9 @@
 // S <- Diag(gC) S + K'^T (U' - W S) becomes S <- Diag(gC) S + N S + b: one
 // tensor-core product per chunk on the serial path.
 //
-// scan_tc_kernel: one CTA per (head, 32-column slice of d_v), serial over the
-// chunks of its range.  Per chunk: D_S = N S (M = 128, the chain), then
+// scan_tc_kernel<W>: one CTA per (head, W 32-column slices of d_v; W = 1, or 2 when
+// one slice per CTA would need more than one wave of SMs), serial over the chunks of
+// its range.  Per chunk: D_S = N S (M = 128, the chain), then
 // S <- Diag(gC) S + D_S + b in fp32 registers (one d_k row per thread; the fp16
 // copy is the next B operand); off the chain, D_O = Qe S (M = 64) and
 // O = D_O + PU'.  A producer warp streams the per-chunk blocks with bulk async
