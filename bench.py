@@ -352,7 +352,7 @@ def build_op(args, cfg, ops, torch, dev, stream, rank):
                   abytes=th * per + B * H * cfg.dk * cfg.dv * 4 * (2 if cfg.s0_std > 0 else 1),
                   flops=3.0 * algorithmic_flops(cfg), tokens=B * T,
                   metric=f"tokens/s FG²-GDN chunked bwd (T={T}, d={cfg.dk}, chunk {chunk}), 1 B200",
-                  e2e_in=None, e2e_out=None, kernel="gdn_chunk_bwd")
+                  e2e_in=None, e2e_out=None, kernel="gdn_chunk_bwd", chunk=chunk)
 
     out = torch.empty((B, T, H, cfg.dv), dtype=dt, device=dev)
     Sf = torch.empty((B, H, cfg.dk, cfg.dv), dtype=torch.float32, device=dev)
@@ -543,7 +543,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic (seeded numpy draws with the workload's distributions)",
             "config": {"workload": cfg.name, "op": args.op, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk,
-                       "dv": cfg.dv, "chunk": cfg.chunk, "per_rank": "one replica per GPU",
+                       "dv": cfg.dv, "chunk": getattr(op, "chunk", cfg.chunk), "per_rank": "one replica per GPU",
                        "l2": f"inputs larger than L2 ({abytes / 1e9:.2f} GB per step vs {L2_BYTES / 2**20:.0f} MiB)"},
             "roofline": roof,
             "e2e": e2e if e2e is not None else {"value": None, "unit": "tokens/s",
