@@ -548,7 +548,8 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
 template <typename Tin, int NR, int NI>
 cudaError_t launch_rev(const Problem& p, const Grads& gr, cudaStream_t stream) {
     const size_t s3 = rev_smem(p.C, p.dk);
-    cudaFuncSetAttribute(rev_scan_kernel<Tin, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+    const cudaError_t e = cudaFuncSetAttribute(rev_scan_kernel<Tin, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+    if (e != cudaSuccess) return e;
     rev_scan_kernel<Tin, NR, NI><<<dim3(p.dv / kNS, p.B * p.H), NT, s3, stream>>>(p, gr);
     return cudaGetLastError();
 }
@@ -566,7 +567,8 @@ cudaError_t launch_rev_nr(const Problem& p, const Grads& gr, cudaStream_t stream
 template <typename Tin, int RPT>
 cudaError_t launch_grad(const Problem& p, const Grads& gr, cudaStream_t stream) {
     const size_t s4 = grad_smem(p.C, p.dk, p.dv);
-    cudaFuncSetAttribute(grad_chunk_kernel<Tin, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
+    const cudaError_t e = cudaFuncSetAttribute(grad_chunk_kernel<Tin, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
+    if (e != cudaSuccess) return e;
     grad_chunk_kernel<Tin, RPT><<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
     return cudaGetLastError();
 }

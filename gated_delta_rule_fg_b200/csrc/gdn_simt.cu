@@ -414,7 +414,8 @@ bool simt_supported(int C, int dk, int dv) {
 
 template <typename Tout, int NR, int NI>
 cudaError_t launch_scan_nr_ni(const Problem& p, dim3 grid, size_t smem, cudaStream_t stream) {
-    cudaFuncSetAttribute(scan_simt_kernel<Tout, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<Tout, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     scan_simt_kernel<Tout, NR, NI><<<grid, kSimtThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
@@ -444,10 +445,14 @@ cudaError_t launch_simt_intra(const Problem& p, bool bf16, cudaStream_t stream) 
     if (p.NC > 0) {
         dim3 g1(p.NC, p.B * p.H);
         if (bf16) {
-            cudaFuncSetAttribute(intra_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+            const cudaError_t e = cudaFuncSetAttribute(intra_simt_kernel<__nv_bfloat16>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+            if (e != cudaSuccess) return e;
             intra_simt_kernel<__nv_bfloat16><<<g1, kSimtThreads, s1, stream>>>(p);
         } else {
-            cudaFuncSetAttribute(intra_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+            const cudaError_t e = cudaFuncSetAttribute(intra_simt_kernel<float>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+            if (e != cudaSuccess) return e;
             intra_simt_kernel<float><<<g1, kSimtThreads, s1, stream>>>(p);
         }
         return cudaGetLastError();
