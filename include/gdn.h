@@ -54,8 +54,12 @@
  *     thread enqueues on the same device is not supported.
  *   - Arguments are validated before anything is enqueued; on an error
  *     nothing is enqueued.  Errors found on the device (a bounded wait that
- *     ran out, a value outside the fp16 operand range) are recorded in the
- *     workspace and read with gdn_workspace_status().
+ *     ran out) are recorded in the workspace and read with
+ *     gdn_workspace_status().
+ *   - The tensor-core path rounds its operands to fp16 (largest finite value
+ *     65504).  The kernels do not check that range: a state whose entries
+ *     exceed it (for instance from an S0 that large) gives undefined numbers,
+ *     as out-of-range alpha and beta do.
  */
 #ifndef GDN_B200_H
 #define GDN_B200_H
@@ -74,7 +78,7 @@ typedef enum {
     GDN_ERR_CUDA = 3,          /* a CUDA launch or copy failed (cudaGetLastError is left set) */
     GDN_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out; outputs are not valid */
     GDN_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or smaller than required */
-    GDN_ERR_RANGE = 6          /* device side: a state or value exceeded the fp16 operand range */
+    GDN_ERR_RANGE = 6          /* reserved: the present kernels do not test the fp16 operand range */
 } gdn_status_t;
 
 typedef enum {
