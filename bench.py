@@ -191,7 +191,8 @@ def cpu_baseline(cfg, target_s: float = 12.0):
     workload, as many as fit in about target_s seconds, one head per thread."""
     import oracle
     threads = oracle.max_threads()
-    x = make_inputs(cfg, T=min(cfg.T, 2048), H=1, B=1)
+    x1_T = min(cfg.T, 2048)
+    x = make_inputs(cfg, T=x1_T, H=1, B=1)
     t0 = time.perf_counter()
     if cfg.deltaproduct_nh:
         oracle.deltaproduct_seq(x["q"], x["k"], x["v"], x["gamma"], x["beta"], x["S0"], nthreads=1)
@@ -199,6 +200,7 @@ def cpu_baseline(cfg, target_s: float = 12.0):
         oracle.gdn_seq(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
                        alpha_scalar=cfg.alpha_scalar, beta_scalar=cfg.beta_scalar, nthreads=1)
     per_tok_head = (time.perf_counter() - t0) / x["q"].shape[1]
+    one_core = 1.0 / (per_tok_head * cfg.H)        # tokens/s (all H heads) on one core
     # heads run in parallel, one per thread; pick a sample of whole heads that fits target_s
     nheads = max(1, min(cfg.B * cfg.H, threads))
     T_s = int(max(256, min(cfg.T, target_s / max(per_tok_head, 1e-9))))
@@ -215,6 +217,10 @@ def cpu_baseline(cfg, target_s: float = 12.0):
     tokens_per_s = token_heads / dt / cfg.H     # tokens/s counts B*T with all H heads
     return {"value": tokens_per_s, "unit": "tokens/s", "cores": min(threads, H_s), "kind": "oracle",
             "sample": f"{H_s} head(s) x {T_s} tokens of {cfg.name} (fp64 C oracle, one head per thread)",
+            "one_core_value": one_core,
+            "one_core_sample": f"1 head x {x1_T} tokens of {cfg.name} on one thread",
+            "nproc": os.cpu_count(), "cpu_model": oracle.host_cpu(),
+            "build": "gcc -O3 -march=native -fopenmp",
             "seconds": dt}
 
 

@@ -65,14 +65,21 @@ size_t workspace_bytes_for(const Problem& p, bool bf16) {
     return kHeaderBytes + inter;
 }
 
-gdn_status_t run(Problem& p, bool bf16, void* workspace, size_t workspace_bytes,
-                 cudaStream_t stream) {
+// Pointer checks shared by the forward entry points (NULL token tensors, 16-byte alignment).
+gdn_status_t check_pointers(const Problem& p) {
     const bool has_tokens = p.B > 0 && p.H > 0 && p.T > 0;
     if (has_tokens && (!p.q || !p.k || !p.v || !p.alpha || !p.beta || !p.out)) return GDN_ERR_INVALID_ARG;
     if (!aligned16(p.q) || !aligned16(p.k) || !aligned16(p.v) || !aligned16(p.alpha) ||
         !aligned16(p.beta) || !aligned16(p.beta_v) || !aligned16(p.out) || !aligned16(p.S0) ||
         !aligned16(p.S_final))
         return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+gdn_status_t run(Problem& p, bool bf16, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+    const gdn_status_t pst = check_pointers(p);
+    if (pst != GDN_OK) return pst;
     const size_t need = workspace_bytes_for(p, bf16);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return GDN_ERR_WORKSPACE;
@@ -90,6 +97,21 @@ int launches_for(const Problem& p, bool bf16) {
 }
 
 }  // namespace
+
+namespace gdn {
+// Every check gdn_chunk_fwd makes before it enqueues work, except the workspace ones.
+gdn_status_t chunk_fwd_check_args(const void* q, const void* k, const void* v, const float* alpha,
+                                  const float* beta, const float* S0, const void* out,
+                                  const float* S_final, int B, int H, int T, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype, unsigned flags) {
+    Problem p;
+    gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false);
+    if (st != GDN_OK) return st;
+    p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta;
+    p.S0 = S0; p.out = const_cast<void*>(out); p.S_final = const_cast<float*>(S_final);
+    return check_pointers(p);
+}
+}  // namespace gdn
 
 extern "C" {
 

@@ -13,13 +13,29 @@
 //   - Set-up: the first call on a device looks up the array's device address with
 //     that device current (cudaGetSymbolAddress) and caches it; in host code the
 //     array's name is only a host-side stand-in, never a device address.  Make the
-//     first call on each device before any stream capture.
+//     first call on each device before any stream capture.  The cache is keyed on
+//     the device's current CUDA context (its context id), so after a
+//     cudaDeviceReset the next call looks the address up again instead of using
+//     an address of the destroyed context.
+//   - Arguments are validated before anything is enqueued: a call rejected with an
+//     error has queued no work.
 //   - Every call shares the array and it keeps the last call's contents; the
-//     status word at its start is cleared on each call.  Calls whose kernels can
-//     overlap on the GPU (other streams, other threads) race on the array.
+//     status word at its start is cleared on each call, and device-side errors
+//     recorded there are not reported back (callers of this entry point have no
+//     workspace to pass to gdn_workspace_status).  Calls whose kernels can overlap
+//     on the GPU (other streams, other threads) race on the array.
 #include <mutex>
 
+#include <cuda.h>
+
 #include "gdn.h"
+
+namespace gdn {
+gdn_status_t chunk_fwd_check_args(const void* q, const void* k, const void* v, const float* alpha,
+                                  const float* beta, const float* S0, const void* out,
+                                  const float* S_final, int B, int H, int T, int dk, int dv, int chunk,
+                                  gdn_dtype_t dtype, unsigned flags);
+}
 
 namespace {
 
@@ -28,20 +44,52 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void* g_scratch_addr[kMaxDevices] = {};
+struct ScratchSlot {
+    void* addr = nullptr;
+    unsigned long long ctx = 0;      // id of the context the address belongs to (0: unknown)
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context, or 0 if it cannot be read.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        looked_up = true;
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, nullptr) == cudaSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, nullptr) == cudaSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+            get_id = reinterpret_cast<CtxGetIdFn>(f2);
+        }
+    }
+    if (!get_current || !get_id) return 0;
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 gdn_status_t scratch_for_current_device(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    ScratchSlot& s = g_scratch[dev];
+    const unsigned long long ctx = current_context_id();
+    if (!s.addr || (ctx != 0 && ctx != s.ctx)) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return GDN_ERR_CUDA;
-        g_scratch_addr[dev] = ptr;
+        s.addr = ptr;
+        s.ctx = current_context_id();     // the lookup makes the context current if it was not
     }
-    *out = g_scratch_addr[dev];
+    *out = s.addr;
     return GDN_OK;
 }
 
@@ -53,10 +101,12 @@ extern "C" gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, cons
                                               int B, int H, int T, int dk, int dv, int chunk,
                                               gdn_dtype_t dtype, unsigned flags,
                                               cudaStream_t stream) {
+    // validation first: nothing is enqueued for a call that is rejected
+    const gdn_status_t chk = gdn::chunk_fwd_check_args(q, k, v, alpha, beta, S0, out, S_final, B, H, T,
+                                                       dk, dv, chunk, dtype, flags);
+    if (chk != GDN_OK) return chk;
     const size_t need = gdn_chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype, flags);
-    if (need == 0)      // invalid or unsupported sizes: let the regular entry point name the error
-        return gdn_chunk_fwd(q, k, v, alpha, beta, S0, out, S_final, B, H, T, dk, dv, chunk, dtype,
-                             flags, nullptr, 0, stream);
+    if (need == 0) return GDN_ERR_UNSUPPORTED;
     if (need > kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;
     void* scratch = nullptr;
     const gdn_status_t st = scratch_for_current_device(&scratch);

@@ -1091,7 +1091,8 @@ int tc_launches(const Problem& p) { return p.NC > 0 ? 2 * tc_segments(p) : 1; }
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
                : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
-    cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+    cudaError_t ae = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+    if (ae != cudaSuccess) return ae;
     // scan width: two slices per CTA when one slice per CTA would take more than one wave
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -1100,7 +1101,8 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto scan = w2 ? tc::scan_tc_kernel<2> : tc::scan_tc_kernel<1>;
     const uint32_t scan_smem = w2 ? tc::ScanCfg<2>::kSmem : tc::ScanCfg<1>::kSmem;
     const int scan_threads = w2 ? tc::ScanCfg<2>::kThreads : tc::ScanCfg<1>::kThreads;
-    cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    ae = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (ae != cudaSuccess) return ae;
     const dim3 g2(tc::J / (w2 ? 2 : 1), p.B * p.H);
     const int P = tc_segments(p);
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream

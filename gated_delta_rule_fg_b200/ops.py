@@ -218,6 +218,8 @@ def chunk_fwd_noalloc(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=F
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if S_final is None and want_state:
         S_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.dtype)
+    _check(S_final, "S_final", torch.float32)
     st = lib().gdn_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
                                      _ptr(out), _ptr(S_final), B, H, T, dk, dv, chunk, code, flags,
                                      _stream(stream))

@@ -123,12 +123,14 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
  * array): every GPU on which the library's device code is loaded holds it until
  * the process exits.  Sizes whose gdn_chunk_fwd_workspace_size exceeds 64 MiB
  * (67108864 bytes) return GDN_ERR_WORKSPACE before anything is enqueued; other
- * argument errors are reported as by gdn_chunk_fwd.  The first call on a device
- * looks up the array's device address (with that device current) and caches it;
- * make that first call before any stream capture.  All calls share the array
- * and it keeps the last call's contents (its status word is cleared at the start
- * of each call, device-side errors are not reported back); calls whose work can
- * overlap on the GPU (different streams or threads) race on it. */
+ * argument errors are reported as by gdn_chunk_fwd, also before anything is
+ * enqueued.  The first call on a device looks up the array's device address
+ * (with that device current) and caches it per device and CUDA context (after a
+ * cudaDeviceReset the next call looks it up again); make that first call before
+ * any stream capture.  All calls share the array and it keeps the last call's
+ * contents (its status word is cleared at the start of each call, device-side
+ * errors are not reported back); calls whose work can overlap on the GPU
+ * (different streams or threads) race on it. */
 gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
                                    const float* alpha, const float* beta,
                                    const float* S0, void* out, float* S_final,

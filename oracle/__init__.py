@@ -31,7 +31,7 @@ Contents and what pins each part (the pins live in tests/test_oracle_*.py):
                      transformed transition, and the two algorithms' agreement
                      (tests/test_oracle_gdn2_pins.py).
 """
-from ._lib import build, deltaproduct_seq, gdn_seq, max_threads  # noqa: F401
+from ._lib import build, deltaproduct_seq, gdn_seq, host_cpu, max_threads  # noqa: F401
 from .chunked import gdn_chunked  # noqa: F401
 from . import spectral  # noqa: F401
 from . import gdn2  # noqa: F401

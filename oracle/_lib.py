@@ -14,18 +14,47 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdn_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
-_SO = os.path.join(_BUILD, "libgdn_oracle.so")
 _lib = None
 
 
+def host_cpu() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _so_path() -> str:
+    """The library is built with -march=native, so its file name carries a hash of the host
+    CPU's model and feature flags: a copy built on another machine is never loaded."""
+    import hashlib
+    ident = host_cpu()
+    try:
+        with open("/proc/cpuinfo") as f:
+            flags = next((l for l in f if l.startswith("flags")), "")
+        ident += flags
+    except OSError:
+        pass
+    tag = hashlib.sha256(ident.encode()).hexdigest()[:12]
+    return os.path.join(_BUILD, f"libgdn_oracle_{tag}.so")
+
+
 def build(force: bool = False) -> str:
-    """Compile gdn_oracle.c into oracle/_build/libgdn_oracle.so (gcc, OpenMP)."""
+    """Compile gdn_oracle.c into oracle/_build/ (gcc -O3 -march=native, OpenMP)."""
+    so = _so_path()
     os.makedirs(_BUILD, exist_ok=True)
-    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
-        tmp = _SO + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _SO)
-    return _SO
+    if force or not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(_SRC):
+        tmp = so + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O3", "-march=native", "-fopenmp", "-shared", "-fPIC", "-o", tmp,
+                               _SRC, "-lm"])
+        os.replace(tmp, so)
+    return so
 
 
 def lib():
