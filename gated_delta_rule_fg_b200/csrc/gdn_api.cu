@@ -41,7 +41,7 @@ gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int d
                           gdn_dtype_t dtype, unsigned flags, bool dp, bool plus = false) {
     if (B < 0 || H < 0 || T < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
-    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR)) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR | GDN_SINGLE_STREAM)) return GDN_ERR_INVALID_ARG;
     if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
     if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
     if (dp && (nh < 1 || nh > 4)) return GDN_ERR_UNSUPPORTED;
@@ -57,6 +57,7 @@ gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int d
     p.alpha_scalar = dp ? 1 : ((flags & GDN_ALPHA_SCALAR) ? 1 : 0);
     p.beta_scalar = beta_scalar ? 1 : 0;
     p.dp = dp ? 1 : 0;
+    p.single_stream = (flags & GDN_SINGLE_STREAM) ? 1 : 0;
     return GDN_OK;
 }
 
@@ -206,7 +207,7 @@ gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
 size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chunk,
                                      gdn_dtype_t dtype, unsigned flags) {
     Problem p;
-    if (flags & ~(unsigned)GDN_ALPHA_SCALAR) return 0;
+    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_SINGLE_STREAM)) return 0;
     if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true) != GDN_OK) return 0;
     if (tc_supported(p, dtype == GDN_BF16)) return kHeaderBytes + tc_inter_bytes(p);
     if (simt_intra_smem_bytes(chunk, dk, dv, true) > 227 * 1024) return 0;
@@ -229,7 +230,7 @@ gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const f
                             gdn_dtype_t dtype, unsigned flags, int mode,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     Problem p;
-    if (flags & ~(unsigned)GDN_ALPHA_SCALAR) return GDN_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_SINGLE_STREAM)) return GDN_ERR_INVALID_ARG;
     if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
     gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
     if (st != GDN_OK) return st;

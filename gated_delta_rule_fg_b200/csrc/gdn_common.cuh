@@ -52,6 +52,7 @@ struct Problem {
     int NC;                 // chunks per sequence = ceil(L / C)
     int alpha_scalar, beta_scalar;
     int dp;                 // 1: DeltaProduct row mapping
+    int single_stream;      // 1: all work on the caller's stream (no side-stream fork)
     int* status;            // workspace header word
     void* inter;            // per-chunk intermediates written by the intra role
     float* S_chunks;        // backward recompute: state at every chunk start,

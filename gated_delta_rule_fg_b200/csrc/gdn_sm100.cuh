@@ -25,6 +25,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// max that propagates NaN (a running max of |x| then reports a NaN input as out of range)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -100,6 +107,29 @@ __device__ __forceinline__ void bulk_g2s(void* smem_dst, const void* gmem_src, u
         : "memory");
 }
 
+// ---------------------------------------------------------------- tensor-map (TMA) loads (no multicast)
+// One box of a 4-D tensor map into shared memory; completion is counted on `bar` (complete_tx).
+// `map` is the address of a __grid_constant__ CUtensorMap kernel parameter.
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const void* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(void* smem_dst, const void* map, int c0, int c1, int c2, int c3, int c4,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const void* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // ---------------------------------------------------------------- per-thread async copies
 // 16-byte global -> shared copy that bypasses registers (L2 only); completes at cp_async_wait_all.
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
@@ -138,6 +168,29 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
     d |= (uint64_t)1 << 46;          // descriptor version of sm_100; base offset 0, no swizzle
     return d;
+}
+
+// 128-byte-swizzled operand (the layout a TMA load with SWIZZLE_128B writes).  A box has rows of
+// 64 16-bit elements (128 B); row r of a box sits at (r / 8) * 1024 + (r % 8) * 128 and its 16-byte
+// chunk j at chunk position j ^ (r % 8); boxes start on 1024-byte boundaries.
+//   K-major (rows = M or N index, elements = K): SBO = 1024 (8-row groups), LBO unused; a K step
+//     of 16 moves the start address by 32 B inside the box, and k >= 64 starts in the next box.
+//   MN-major (rows = K index, elements = M or N): SBO = 1024 (8-row groups along K), LBO = the
+//     stride between boxes along M/N; a K step of 16 moves the start address by 2048 B.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;          // SWIZZLE_128B
+    return d;
+}
+// Byte offset of element (row, col) of a tile stored as 128-byte-swizzled boxes of 64 columns,
+// the boxes `box_stride` bytes apart.
+__host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t col, uint32_t box_stride) {
+    return (col >> 6) * box_stride + (row >> 3) * 1024u + (row & 7u) * 128u +
+           ((((col & 63u) >> 3) ^ (row & 7u)) << 4) + (col & 7u) * 2u;
 }
 
 // kind::f16 instruction descriptor: fp16 A and B, fp32 accumulator.

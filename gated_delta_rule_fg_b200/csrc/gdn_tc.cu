@@ -31,38 +31,12 @@
 // the caller's stream while the scan of range s runs on the side stream.
 #include <mutex>
 
-#include "gdn_common.cuh"
-#include "gdn_sm100.cuh"
+#include "gdn_tc_common.cuh"
 
 namespace gdn {
 using namespace sm100;
 
 namespace tc {
-
-constexpr int C = 64;          // chunk
-constexpr int D = 128;         // dk = dv
-constexpr int NT = 256;        // intra threads
-constexpr int NS = 32;         // scan: columns per CTA
-constexpr int J = D / NS;      // scan: slices per head
-constexpr float kMaxHalfSpan = 6.0f;
-
-// Per (head, chunk) block in the workspace (bytes), written by the intra kernel and read
-// by the scan kernel.  "sw" rows: 32 fp16 per row, the four 16-byte groups of row x are
-// stored in the order g ^ ((x >> 1) & 3), so eight consecutive rows read as 16-byte
-// vectors hit eight different bank groups.
-constexpr uint32_t kOffN = 0;            // N = -K'^T W, fp16 128x128, K-major (m=i, k=c): SBO 2048, LBO 128
-constexpr uint32_t kOffQe = 32768;       // Qe fp16 64x128, MN-major (m=r, k=c): SBO 2048, LBO 128
-constexpr uint32_t kOffB = 49152;        // b = K'^T U', fp16 [J][128][NS] (sw rows)
-constexpr uint32_t kOffPU = 81920;       // PU', fp16 [J][64][NS] (sw rows)
-constexpr uint32_t kOffGC = 98304;       // e^{g_last}, fp32 [128]
-constexpr uint32_t kOffKp = 98816;       // K' fp16 (m=i, k=r), MN-major SBO 1024 LBO 128 (intra's own scratch)
-constexpr uint32_t kBlockBytes = 115200;
-// Fallback chunks (element-wise A and P) stage q^ (fp16) in the N area, k~ (fp16) in the
-// PU' area and g (fp32) in the b area; those areas are written only afterwards.
-
-__host__ __device__ __forceinline__ uint32_t sw_half(uint32_t row, uint32_t j) {
-    return row * NS + 8u * (((j >> 3) ^ ((row >> 1) & 3u))) + (j & 7u);
-}
 
 // intra shared memory map (bytes)
 constexpr uint32_t kR0 = 0;              // [KG; QG] fp16 K-major (row, ch): SBO 2048, LBO 128  -> later W~^T (K-major (ch, row): SBO 128, LBO 2048)
@@ -85,46 +59,6 @@ static_assert(2 * (kIntraSmem + 1024) <= 228 * 1024, "two intra CTAs per SM (1 K
 
 constexpr uint32_t kTmemCols = 256;
 // TMEM columns: D0 / D3 at 0, D1 (W~^T) at 64, D2 (U'^T) at 128, D4 (PU'^T) at 192.
-
-// swizzled fp32 64x64: element (r, i)
-__device__ __forceinline__ int sw64(int r, int i) { return r * 64 + ((((i >> 2) ^ (r & 15))) << 2) + (i & 3); }
-
-// sqrt(x) for x >= 0 as x * rsqrt(x): a few ulp in fp32, far below the fp16 rounding of the
-// operands it scales, and shorter than the IEEE-rounded square root (x = 0 gives 0).
-__device__ __forceinline__ float sqrt_op(float x) { return x > 0.f ? x * rsqrtf(x) : 0.f; }
-
-__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-__device__ __forceinline__ float4 ldg16f(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
-
-__device__ __forceinline__ void bf8_to_f(const uint4 u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
-__device__ __forceinline__ uint4 f_to_h8(const float* f) {
-    uint4 u;
-    __half2 h0 = __floats2half2_rn(f[0], f[1]);
-    __half2 h1 = __floats2half2_rn(f[2], f[3]);
-    __half2 h2 = __floats2half2_rn(f[4], f[5]);
-    __half2 h3 = __floats2half2_rn(f[6], f[7]);
-    u.x = *reinterpret_cast<uint32_t*>(&h0);
-    u.y = *reinterpret_cast<uint32_t*>(&h1);
-    u.z = *reinterpret_cast<uint32_t*>(&h2);
-    u.w = *reinterpret_cast<uint32_t*>(&h3);
-    return u;
-}
-
-__device__ __forceinline__ void st16(uint8_t* base, uint32_t off, uint4 v) {
-    *reinterpret_cast<uint4*>(base + off) = v;
-}
-
-__device__ __forceinline__ void record_timeout(int* status) {
-    atomicCAS(status, kDevOk, kDevTimeout);
-}
 
 // ============================================================================ intra
 // kPlus: FG^2-GDN+ (separate value rate beta^v, eq. (13)).
@@ -941,8 +875,11 @@ __global__ void __launch_bounds__(ScanCfg<W>::kThreads, 1) scan_tc_kernel(Proble
         const int j0 = (slice0 + sl) * NS;                     // first state column of this warp
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         float S[NS];
+        float smax = 0.f;
 #pragma unroll
         for (int j = 0; j < NS; ++j) S[j] = S_in ? S_in[((size_t)bh * D + row) * D + j0 + j] : 0.f;
+#pragma unroll
+        for (int j = 0; j < NS; ++j) smax = fmax_nan(smax, fabsf(S[j]));
 #pragma unroll
         for (int j = 0; j < NS; j += 8) st16(sm + Cfg::kSop, off_mnmajor(NS * sl + j, row, 2048, 128), f_to_h8(S + j));
         fence_async_smem();
@@ -982,7 +919,14 @@ __global__ void __launch_bounds__(ScanCfg<W>::kThreads, 1) scan_tc_kernel(Proble
                 mbar_arrive(s_ready);                          // this warp's part of S_{ch+1} is in Sop
                 mbar_arrive(&emptyNB[s3]);
             }
+            // largest |S| entry so far (off the chain: nothing waits for it); above the fp16
+            // range the fp16 copy, and so the result, is not valid
+#pragma unroll
+            for (int j = 0; j < NS; ++j) smax = fmax_nan(smax, fabsf(S[j]));
         }
+        // NaN compares false: a NaN state is reported too
+        if (ok && __any_sync(0xffffffffu, !(smax <= 65504.f)) && lane == 0)
+            atomicCAS(p.status, kDevOk, kDevRange);
         if (!ok) {
             if (lane == 0) record_timeout(p.status);
         } else if (S_out) {
@@ -1088,11 +1032,25 @@ size_t tc_inter_bytes(const Problem& p) {
 int tc_launches(const Problem& p) { return p.NC > 0 ? 2 * tc_segments(p) : 1; }
 
 
+// gdn_tc2.cu: the TMA-fed intra role, for the problems it covers
+bool tc2_usable(const Problem& p);
+cudaError_t launch_intra_tma(const Problem& p, int cb, int n, cudaStream_t stream);
+
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
                : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
-    cudaError_t ae = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
-    if (ae != cudaSuccess) return ae;
+    const bool tma = tc2_usable(p);
+    cudaError_t ae = cudaSuccess;
+    if (!tma) {
+        ae = cudaFuncSetAttribute(intra, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::kIntraSmem);
+        if (ae != cudaSuccess) return ae;
+    }
+    // intra role over chunks [cb, cb + n) of every head
+    auto launch_intra = [&](int cb, int n, cudaStream_t st) -> cudaError_t {
+        if (tma) return launch_intra_tma(p, cb, n, st);
+        intra<<<dim3(n, p.B * p.H), tc::NT, tc::kIntraSmem, st>>>(p, cb);
+        return cudaGetLastError();
+    };
     // scan width: two slices per CTA when one slice per CTA would take more than one wave
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -1106,13 +1064,12 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     const dim3 g2(tc::J / (w2 ? 2 : 1), p.B * p.H);
     const int P = tc_segments(p);
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream
-        intra<<<dim3(p.NC, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(p, 0);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_intra(0, p.NC, stream);
         if (e != cudaSuccess) return e;
         scan<<<g2, scan_threads, scan_smem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
         return cudaGetLastError();
     };
-    if (P == 1) return one_stream();
+    if (P == 1 || p.single_stream) return one_stream();
     std::unique_lock<std::mutex> lock;
     SideStream* side = side_stream_lock(lock);
     if (!side) return one_stream();
@@ -1124,8 +1081,7 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     for (int sg = 0; sg < P && e == cudaSuccess; ++sg) {
         int cb, ce;
         seg_range(p.NC, P, sg, cb, ce);
-        intra<<<dim3(ce - cb, p.B * p.H), tc::NT, tc::kIntraSmem, stream>>>(p, cb);
-        e = cudaGetLastError();
+        e = launch_intra(cb, ce - cb, stream);
         if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.ready[sg], 0);
         if (e != cudaSuccess) break;

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, 1, 2, 3
 GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE, GDN_ERR_RANGE = 4, 5, 6
 GDN_F32, GDN_BF16 = 0, 1
-GDN_ALPHA_SCALAR, GDN_BETA_SCALAR = 1, 2
+GDN_ALPHA_SCALAR, GDN_BETA_SCALAR, GDN_SINGLE_STREAM = 1, 2, 4
 
 # Every symbol include/gdn.h declares, with its ctypes signature.
 _P = ctypes.c_void_p
@@ -139,7 +139,7 @@ def alloc_workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def chunk_fwd(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=False, beta_scalar=False,
-              out=None, S_final=None, want_state=True, workspace=None, stream=None):
+              out=None, S_final=None, want_state=True, workspace=None, stream=None, single_stream=False):
     """FG^2-GDN chunkwise forward through gdn_chunk_fwd.
 
     q, k [B,T,H,dk], v [B,T,H,dv] (bf16 or float32, same dtype); alpha/beta float32
@@ -153,7 +153,8 @@ def chunk_fwd(q, k, v, alpha, beta, S0=None, *, chunk=64, alpha_scalar=False, be
         _check(t, n, q.dtype)
     for t, n in ((alpha, "alpha"), (beta, "beta"), (S0, "S0")):
         _check(t, n, torch.float32)
-    flags = (GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+    flags = ((GDN_ALPHA_SCALAR if alpha_scalar else 0) | (GDN_BETA_SCALAR if beta_scalar else 0)
+             | (GDN_SINGLE_STREAM if single_stream else 0))
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
     if S_final is None and want_state:

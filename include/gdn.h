@@ -44,7 +44,8 @@
  *     `workspace` (device memory, 256-byte aligned, at least the size the
  *     matching *_workspace_size function returns); one workspace must not be
  *     used by two calls that can run at the same time.  The library allocates
- *     no device memory.  For long sequences on the tensor-core path it keeps,
+ *     no device memory.  Unless GDN_SINGLE_STREAM is given, for long sequences
+ *     on the tensor-core path it keeps,
  *     per device and created on first use, one high-priority stream and a few
  *     events: a call then forks onto that stream (so part of its work overlaps)
  *     and joins back before returning, so all of its work is still ordered
@@ -88,7 +89,10 @@ typedef enum {
 
 enum {
     GDN_ALPHA_SCALAR = 1u,     /* alpha is one value per token and head: [B,T,H] (GDN) */
-    GDN_BETA_SCALAR = 2u       /* beta is one value per token and head: [B,T,H] (KDA, GDN, DeltaNet) */
+    GDN_BETA_SCALAR = 2u,      /* beta is one value per token and head: [B,T,H] (KDA, GDN, DeltaNet) */
+    GDN_SINGLE_STREAM = 4u     /* keep all of the call's work on `stream`: no fork onto the library's
+                                  per-device side stream (no lock, no global state is touched); the
+                                  result is the same bit for bit, long sequences take longer */
 };
 
 /* Bytes of workspace gdn_chunk_fwd needs for these sizes (0 if the sizes are
@@ -220,7 +224,7 @@ size_t gdn2_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int ch
  * chunk's prep; the chunk form is the non-tied WY form (A pairs erase with write
  * vectors, the state is read along j' and written along k^).
  *   q, k [B,T,H,dk], v, out [B,T,H,dv]: dtype storage; alpha float32 [B,T,H,dk] (or
- *   [B,T,H] with GDN_ALPHA_SCALAR, the only flag); eta float32 [B,T,H] (>= 0);
+ *   [B,T,H] with GDN_ALPHA_SCALAR; GDN_SINGLE_STREAM is the only other flag); eta float32 [B,T,H] (>= 0);
  *   b_gate float32 [B,T,H,dk] in [0,1]; S0, S_final float32 [B,H,dk,dv] (may be NULL).
  * GDN_BF16 with chunk 64 and dk == dv == 128 runs on the tensor-core path (fp16
  * operands, as gdn_chunk_fwd); other shapes run on the float32 CUDA-core path with

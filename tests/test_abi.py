@@ -88,6 +88,8 @@ def test_argument_validation_before_launch(L):
     # empty batch: valid, nothing to do, no device access
     assert _call(L, B=0) == ops.GDN_OK
     assert _call(L, H=0) == ops.GDN_OK
+    assert _call(L, B=0, flags=ops.GDN_SINGLE_STREAM) == ops.GDN_OK   # the single-stream flag is accepted
+    assert L.gdn_chunk_fwd_workspace_size(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, ops.GDN_SINGLE_STREAM) > 0
 
 
 def test_deltaproduct_validation(L):

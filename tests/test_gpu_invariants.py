@@ -145,3 +145,19 @@ def test_too_small_workspace_is_rejected_without_launch():
         ops.chunk_fwd(to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt),
                       to_dev(x["alpha"]), to_dev(x["beta"]), None, chunk=64, workspace=ws)
     assert e.value.code == ops.GDN_ERR_WORKSPACE
+
+
+def test_single_stream_flag_same_result():
+    """GDN_SINGLE_STREAM keeps the whole call on the caller's stream (no fork onto the
+    library's side stream); a sequence long enough to be cut into chunk ranges gives the
+    default call's result bit for bit."""
+    ops = _ops()
+    cfg = GdnConfig("single", B=1, H=2, T=64 * 70 + 9, dk=128, dv=128, chunk=64, s0_std=0.05, seed=41)
+    x = make_inputs(cfg)
+    dt = torch.bfloat16
+    args = (to_dev(x["q"], dt), to_dev(x["k"], dt), to_dev(x["v"], dt), to_dev(x["alpha"]), to_dev(x["beta"]),
+            to_dev(x["S0"]))
+    o1, s1 = ops.chunk_fwd(*args, chunk=64)
+    o2, s2 = ops.chunk_fwd(*args, chunk=64, single_stream=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
