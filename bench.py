@@ -89,7 +89,8 @@ def load_traffic(kernel: str, workload: str, source_hash: str):
     return float(e["dram_bytes_per_launch"])
 
 
-TC_SOURCES = ("gdn_tc.cu", "gdn_sm100.cuh")     # the timed kernels' own code
+TC_SOURCES = ("gdn_tc.cu", "gdn_tc2.cu", "gdn_scan2.cu", "gdn_tc_common.cuh",
+              "gdn_sm100.cuh")     # the timed kernels' own code
 
 
 def code_only(text: str) -> str:

@@ -1,6 +1,8 @@
 // gdn_api.cu -- the C ABI declared in include/gdn.h: argument validation,
 // workspace sizing and kernel dispatch.  Every step of the computation runs in
 // the CUDA kernels of this library; there is no host or CPU fallback.
+#include <cstdlib>
+
 #include "gdn.h"
 #include "gdn_common.cuh"
 
@@ -58,6 +60,15 @@ gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int d
     p.beta_scalar = beta_scalar ? 1 : 0;
     p.dp = dp ? 1 : 0;
     p.single_stream = (flags & GDN_SINGLE_STREAM) ? 1 : 0;
+    p.test_skip_chunk = -1;
+    if (const char* e = std::getenv("GDN_TEST_SCAN_SKIP_CHUNK")) {
+        char* end = nullptr;
+        const long c = std::strtol(e, &end, 10);
+        if (end != e && c >= 0 && c < (1L << 30)) {
+            p.test_skip_chunk = (int)c;
+            p.test_wait_ns = 1000000ull;        // 1 ms
+        }
+    }
     return GDN_OK;
 }
 

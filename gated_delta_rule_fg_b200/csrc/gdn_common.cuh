@@ -53,6 +53,12 @@ struct Problem {
     int alpha_scalar, beta_scalar;
     int dp;                 // 1: DeltaProduct row mapping
     int single_stream;      // 1: all work on the caller's stream (no side-stream fork)
+    // Failure-detection test knob (environment variable GDN_TEST_SCAN_SKIP_CHUNK, read per
+    // call; unset in normal use): the tensor-core scan's producer leaves chunk test_skip_chunk
+    // unloaded, so the roles that wait for it run out of their bound, which is then
+    // test_wait_ns instead of the 2 s default.  -1 / 0: off.
+    int test_skip_chunk;
+    unsigned long long test_wait_ns;
     int* status;            // workspace header word
     void* inter;            // per-chunk intermediates written by the intra role
     float* S_chunks;        // backward recompute: state at every chunk start,

@@ -1032,9 +1032,11 @@ size_t tc_inter_bytes(const Problem& p) {
 int tc_launches(const Problem& p) { return p.NC > 0 ? 2 * tc_segments(p) : 1; }
 
 
-// gdn_tc2.cu: the TMA-fed intra role, for the problems it covers
+// gdn_tc2.cu: the TMA-fed intra role, for the problems it covers; gdn_scan2.cu: the scan role
+// for its blocks
 bool tc2_usable(const Problem& p);
 cudaError_t launch_intra_tma(const Problem& p, int cb, int n, cudaStream_t stream);
+cudaError_t launch_scan2(const Problem& p, int cb, int ce, const float* S_in, float* S_out, cudaStream_t stream);
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
@@ -1059,15 +1061,22 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     auto scan = w2 ? tc::scan_tc_kernel<2> : tc::scan_tc_kernel<1>;
     const uint32_t scan_smem = w2 ? tc::ScanCfg<2>::kSmem : tc::ScanCfg<1>::kSmem;
     const int scan_threads = w2 ? tc::ScanCfg<2>::kThreads : tc::ScanCfg<1>::kThreads;
-    ae = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
-    if (ae != cudaSuccess) return ae;
+    if (!tma) {
+        ae = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+        if (ae != cudaSuccess) return ae;
+    }
     const dim3 g2(tc::J / (w2 ? 2 : 1), p.B * p.H);
     const int P = tc_segments(p);
+    // scan role over chunks [cb, ce)
+    auto launch_scan = [&](int cb, int ce, const float* S_in, float* S_out, cudaStream_t st) -> cudaError_t {
+        if (tma) return launch_scan2(p, cb, ce, S_in, S_out, st);
+        scan<<<g2, scan_threads, scan_smem, st>>>(p, cb, ce, S_in, S_out);
+        return cudaGetLastError();
+    };
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream
         cudaError_t e = launch_intra(0, p.NC, stream);
         if (e != cudaSuccess) return e;
-        scan<<<g2, scan_threads, scan_smem, stream>>>(p, 0, p.NC, p.S0, p.S_final);
-        return cudaGetLastError();
+        return launch_scan(0, p.NC, p.S0, p.S_final, stream);
     };
     if (P == 1 || p.single_stream) return one_stream();
     std::unique_lock<std::mutex> lock;
@@ -1085,9 +1094,7 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
         if (e == cudaSuccess) e = cudaEventRecord(ss.ready[sg], stream);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.stream, ss.ready[sg], 0);
         if (e != cudaSuccess) break;
-        scan<<<g2, scan_threads, scan_smem, ss.stream>>>(
-            p, cb, ce, sg == 0 ? p.S0 : handoff, sg == P - 1 ? p.S_final : handoff);
-        e = cudaGetLastError();
+        e = launch_scan(cb, ce, sg == 0 ? p.S0 : handoff, sg == P - 1 ? p.S_final : handoff, ss.stream);
     }
     // join: whatever happened above, the caller's stream waits for the side stream's work
     cudaError_t j = cudaEventRecord(ss.join, ss.stream);

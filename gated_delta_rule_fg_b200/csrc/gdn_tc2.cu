@@ -20,8 +20,9 @@
 //   b  =  diag(ref) (Y V)                 (=  K'^T U')
 //   Qe = (QG - Z KG) diag(ref)            (=  Q^ e^g - P W)
 //   PU' = Z V
-// because K' = KI diag(ref) and W = T KG diag(ref).  Three rounds of tensor-core products:
-// [A; P]; then Y and Z; then N, PU'^T and Qe^T, and b once N has left its accumulator.
+// because K' = KI diag(ref) and W = T KG diag(ref).  Four rounds of tensor-core products:
+// [A; P]; Y and Z; N~ and Qe~; b~ and PU'.  Qe is stored K-major (rows of 128 channels), the
+// layout the scan copies into tensor memory as an A operand.
 #include <cuda.h>
 
 #include "gdn_tc_common.cuh"
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const float P = pre[e] * lp[i][e];
-                const float rp = __frcp_rn(P);
+                const float rp = __fdividef(1.f, P);     // P >= gamma >= e^{-12}: no overflow
                 const float sb = tc::sqrt_op(be[i][e]);
                 const float kt = fk[e] * ik[i] * sb;
                 KG[e] = kt * (P * iv[e]);
@@ -446,14 +447,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     // rows of A are broadcast shared-memory reads), then T10 = -T11 (A10 T00) on 16x16 and
     // 32x32 blocks; each merge overwrites the A block it consumed.
     if (warp < 4) {
+        // rows of A read as broadcast float4 (four consecutive entries share one swizzled 16-byte
+        // piece); four partial sums keep the dependent chain of each row short
         const int bb = 16 * warp, jc = lane & 15;
         float t[16];
 #pragma unroll
         for (int r2 = 0; r2 < 16; ++r2) {
-            float acc = (r2 == jc) ? 1.f : 0.f;
+            float acc[4] = {(r2 == jc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < r2; ++i) acc -= A32[tc::sw64(bb + r2, bb + i)] * t[i];
-            t[r2] = acc;
+            for (int i4 = 0; i4 < r2; i4 += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(A32 + tc::sw64(bb + r2, bb + i4));
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (i4 + e < r2) acc[e] = fmaf(-av[e], t[i4 + e], acc[e]);
+            }
+            t[r2] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         }
         __syncwarp();
         if (lane < 16) {
@@ -466,46 +475,68 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
         const int m = tid >> 7, qd = tid & 127;
         const int rw = qd >> 3, j2 = (qd & 7) * 2;
         const int bs = 32 * m;
-        float x0 = 0.f, x1 = 0.f;
+        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float a = A32[tc::sw64(bs + 16 + rw, bs + i)];
-            x0 = fmaf(a, A32[tc::sw64(bs + i, bs + j2)], x0);
-            x1 = fmaf(a, A32[tc::sw64(bs + i, bs + j2 + 1)], x1);
+        for (int i4 = 0; i4 < 16; i4 += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(A32 + tc::sw64(bs + 16 + rw, bs + i4));
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 tv = *reinterpret_cast<const float2*>(A32 + tc::sw64(bs + i4 + e, bs + j2));
+                if (e & 1) { x2 = fmaf(av[e], tv.x, x2); x3 = fmaf(av[e], tv.y, x3); }
+                else       { x0 = fmaf(av[e], tv.x, x0); x1 = fmaf(av[e], tv.y, x1); }
+            }
         }
-        scr[m * 256 + rw * 16 + j2] = x0;
-        scr[m * 256 + rw * 16 + j2 + 1] = x1;
+        *reinterpret_cast<float2*>(scr + m * 256 + rw * 16 + j2) = make_float2(x0 + x2, x1 + x3);
         __syncthreads();
-        float y0 = 0.f, y1 = 0.f;
+        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
 #pragma unroll
-        for (int mm = 0; mm < 16; ++mm) {
-            const float tt = A32[tc::sw64(bs + 16 + rw, bs + 16 + mm)];
-            y0 = fmaf(tt, scr[m * 256 + mm * 16 + j2], y0);
-            y1 = fmaf(tt, scr[m * 256 + mm * 16 + j2 + 1], y1);
+        for (int m4 = 0; m4 < 16; m4 += 4) {
+            const float4 tt = *reinterpret_cast<const float4*>(A32 + tc::sw64(bs + 16 + rw, bs + 16 + m4));
+            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 xv = *reinterpret_cast<const float2*>(scr + m * 256 + (m4 + e) * 16 + j2);
+                if (e & 1) { y2 = fmaf(tv[e], xv.x, y2); y3 = fmaf(tv[e], xv.y, y3); }
+                else       { y0 = fmaf(tv[e], xv.x, y0); y1 = fmaf(tv[e], xv.y, y1); }
+            }
         }
-        A32[tc::sw64(bs + 16 + rw, bs + j2)] = -y0;
-        A32[tc::sw64(bs + 16 + rw, bs + j2 + 1)] = -y1;
+        *reinterpret_cast<float2*>(A32 + tc::sw64(bs + 16 + rw, bs + j2)) = make_float2(-(y0 + y2), -(y1 + y3));
     }
     __syncthreads();
     {   // 32x32 merge: T_BL = -T_BR (A_BL T_TL)
         const int rw = tid >> 3, j4 = (tid & 7) * 4;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            const float a = A32[tc::sw64(32 + rw, i)];
-            const float4 tv = *reinterpret_cast<const float4*>(A32 + tc::sw64(i, j4));
-            x.x = fmaf(a, tv.x, x.x); x.y = fmaf(a, tv.y, x.y); x.z = fmaf(a, tv.z, x.z); x.w = fmaf(a, tv.w, x.w);
+        float4 xa = make_float4(0.f, 0.f, 0.f, 0.f), xb = xa;
+#pragma unroll
+        for (int i4 = 0; i4 < 32; i4 += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(A32 + tc::sw64(32 + rw, i4));
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 tv = *reinterpret_cast<const float4*>(A32 + tc::sw64(i4 + e, j4));
+                float4& x = (e & 1) ? xb : xa;
+                x.x = fmaf(av[e], tv.x, x.x); x.y = fmaf(av[e], tv.y, x.y);
+                x.z = fmaf(av[e], tv.z, x.z); x.w = fmaf(av[e], tv.w, x.w);
+            }
         }
-        *reinterpret_cast<float4*>(scr + 512 + rw * 32 + j4) = x;
+        *reinterpret_cast<float4*>(scr + 512 + rw * 32 + j4) =
+            make_float4(xa.x + xb.x, xa.y + xb.y, xa.z + xb.z, xa.w + xb.w);
         __syncthreads();
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int mm = 0; mm < 32; ++mm) {
-            const float tt = A32[tc::sw64(32 + rw, 32 + mm)];
-            const float4 xv = *reinterpret_cast<const float4*>(scr + 512 + mm * 32 + j4);
-            y.x = fmaf(tt, xv.x, y.x); y.y = fmaf(tt, xv.y, y.y); y.z = fmaf(tt, xv.z, y.z); y.w = fmaf(tt, xv.w, y.w);
+        float4 ya = make_float4(0.f, 0.f, 0.f, 0.f), yb = ya;
+#pragma unroll
+        for (int m4 = 0; m4 < 32; m4 += 4) {
+            const float4 tt = *reinterpret_cast<const float4*>(A32 + tc::sw64(32 + rw, 32 + m4));
+            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float4 xv = *reinterpret_cast<const float4*>(scr + 512 + (m4 + e) * 32 + j4);
+                float4& y = (e & 1) ? yb : ya;
+                y.x = fmaf(tv[e], xv.x, y.x); y.y = fmaf(tv[e], xv.y, y.y);
+                y.z = fmaf(tv[e], xv.z, y.z); y.w = fmaf(tv[e], xv.w, y.w);
+            }
         }
-        *reinterpret_cast<float4*>(A32 + tc::sw64(32 + rw, j4)) = make_float4(-y.x, -y.y, -y.z, -y.w);
+        *reinterpret_cast<float4*>(A32 + tc::sw64(32 + rw, j4)) =
+            make_float4(-(ya.x + yb.x), -(ya.y + yb.y), -(ya.z + yb.z), -(ya.w + yb.w));
     }
     __syncthreads();
     for (int idx = tid; idx < 512; idx += NT) {   // T -> fp16 (rows contiguous in 16-byte pieces)
@@ -574,25 +605,24 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     __syncthreads();
     tc_fence_after();
 
-    // ---------------------------------------------------------------- N~ = Y KG, PU'^T = V^T Z^T, Qe~^T = QG^T - KG^T Z^T
+    // ---------------------------------------------------------------- N~ = Y KG, Qe~ = QG - Z KG
     if (ok) {
         if (tid == 0) {
             const uint32_t idN = idesc_f16(128, 128, false, true);
-            const uint32_t idT = idesc_f16(128, 64, true, false);
-            const uint32_t idTn = idesc_f16(128, 64, true, false, true);
+            const uint32_t idQ = idesc_f16(64, 128, false, true);
+            const uint32_t idQn = idesc_f16(64, 128, false, true, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t aY = sdesc(base + kA32 + kk * 256, 128, 1024);
-                const uint64_t bZ = sdesc(base + kT16 + kk * 256, 128, 1024);
-                mma_f16(t0 + 0, aY, sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024), idN, kk > 0);
-                mma_f16(t0 + 128, sdesc_sw128(base + kV + kk * 2048, 8192, 1024), bZ, idT, kk > 0);
-                mma_f16(t0 + 192, sdesc_sw128(base + kKQ + 8192 + kk * 2048, 16384, 1024),
-                        sdesc(base + kP16 + kk * 256, 128, 1024), idT, kk > 0);
+                const uint64_t bKG = sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024);
+                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), bKG, idN, kk > 0);
+                // Qe~ = I QG - Z KG (M = 64: the identity, then Z, as A; QG and KG as MN-major B)
+                mma_f16(t0 + 128, sdesc(base + kP16 + kk * 256, 128, 1024),
+                        sdesc_sw128(base + kKQ + 8192 + kk * 2048, 16384, 1024), idQ, kk > 0);
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-                mma_f16(t0 + 192, sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024), sdesc(base + kT16 + kk * 256, 128, 1024),
-                        idTn, true);
+                mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024),
+                        idQn, true);
             mma_commit(bar_mma);
         }
         ok = mbar_wait(bar_mma, phase);
@@ -601,69 +631,61 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     ok = __syncthreads_and(ok);
     if (!ok && tid == 0) tc::record_timeout(p.status);
     tc_fence_after();
-    if (ok) {   // N = -diag(row) N~ diag(col) -> block (K-major (m = i, k = c): SBO 2048, LBO 128)
+    if (ok) {
         const int q = warp & 3, chh = warp >> 2;
-        const int cc = 32 * q + lane;
-        const float rs = -trow[cc];
         const uint32_t lb = (uint32_t)(32 * q) << 16;
+        {   // N = -diag(row) N~ diag(col) -> block (K-major (m = i, k = c): SBO 2048, LBO 128)
+            const int cc = 32 * q + lane;
+            const float rs = -trow[cc];
+#pragma unroll 1
+            for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
+                float x[32];
+                tmem_ld32(t0 + lb + c0, x);
+#pragma unroll
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 cs = *reinterpret_cast<const float4*>(tcol + c0 + e4);
+                    x[e4] *= rs * cs.x; x[e4 + 1] *= rs * cs.y; x[e4 + 2] *= rs * cs.z; x[e4 + 3] *= rs * cs.w;
+                }
+#pragma unroll
+                for (int g8 = 0; g8 < 32; g8 += 8)
+                    *reinterpret_cast<uint4*>(blk + tc::kOffN + off_kmajor(cc, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
+            }
+        }
+        // Qe = Qe~ diag(col) (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (K-major
+        // (m = r, k = c): SBO 2048, LBO 128)
 #pragma unroll 1
         for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
             float x[32];
-            tmem_ld32(t0 + lb + c0, x);
+            tmem_ld32(t0 + lb + 128 + c0, x);
+            if (lane < 16) {
+                const int r = 16 * q + lane;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] *= rs * tcol[c0 + e];
+                for (int e4 = 0; e4 < 32; e4 += 4) {
+                    const float4 cs = *reinterpret_cast<const float4*>(tcol + c0 + e4);
+                    x[e4] *= cs.x; x[e4 + 1] *= cs.y; x[e4 + 2] *= cs.z; x[e4 + 3] *= cs.w;
+                }
 #pragma unroll
-            for (int g8 = 0; g8 < 32; g8 += 8)
-                *reinterpret_cast<uint4*>(blk + tc::kOffN + off_kmajor(cc, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
+                for (int g8 = 0; g8 < 32; g8 += 8)
+                    *reinterpret_cast<uint4*>(blk + tc::kOffQe + off_kmajor(r, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // b~ = Y V into the columns N~ used
-    if (ok && tid == 0) {
-        const uint32_t idN = idesc_f16(128, 128, false, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-            mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), sdesc_sw128(base + kV + kk * 2048, 8192, 1024), idN,
-                    kk > 0);
-        mma_commit(bar_mma);
-    }
-    if (ok && warp < 4) {        // Qe = Qe~ diag(col) -> block (MN-major (m = r, k = c): SBO 2048, LBO 128)
-        const int cc = 32 * warp + lane;
-        const float cs = tcol[cc];
-        const uint32_t lb = (uint32_t)(32 * warp) << 16;
-        float x0[32], x1[32];
-        tmem_ld32(t0 + lb + 192, x0);
-        tmem_ld32(t0 + lb + 224, x1);
-#pragma unroll
-        for (int r0 = 0; r0 < C; r0 += 8) {
-            const float* src = (r0 < 32 ? x0 : x1) + (r0 & 31);
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = src[e] * cs;
-            *reinterpret_cast<uint4*>(blk + tc::kOffQe + off_mnmajor(r0, cc, 2048, 128)) = tc::f_to_h8(f);
-        }
-    } else if (ok) {             // PU' slice w-4: assembled in the dead T16 / P16 area, copied out as 16-byte vectors
-        const int sl = warp - 4;
-        const uint32_t lb = (uint32_t)(32 * sl) << 16;
-        float x0[32], x1[32];
-        tmem_ld32(t0 + lb + 128, x0);
-        tmem_ld32(t0 + lb + 160, x1);
-        __half* st = reinterpret_cast<__half*>(sm + kT16 + sl * (C * NS * 2));
-#pragma unroll
-        for (int r2 = 0; r2 < C; ++r2) {
-            const float x = r2 < 32 ? x0[r2] : x1[r2 - 32];
-            vmax = fmax_nan(vmax, fabsf(x));
-            st[tc::sw_half(r2, lane)] = __float2half_rn(x);
-        }
-        __syncwarp();
-        const uint4* srcv = reinterpret_cast<const uint4*>(st);
-        uint4* dstv = reinterpret_cast<uint4*>(blk + tc::kOffPU + sl * (C * NS * 2));
-#pragma unroll
-        for (int i = 0; i < C * NS * 2 / 16 / 32; ++i) dstv[lane + 32 * i] = srcv[lane + 32 * i];
-    }
+    // ---------------------------------------------------------------- b~ = Y V, PU' = Z V
     if (ok) {
+        if (tid == 0) {
+            const uint32_t idN = idesc_f16(128, 128, false, true);
+            const uint32_t idP = idesc_f16(64, 128, false, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bV = sdesc_sw128(base + kV + kk * 2048, 8192, 1024);
+                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), bV, idN, kk > 0);
+                mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), bV, idP, kk > 0);
+            }
+            mma_commit(bar_mma);
+        }
         ok = mbar_wait(bar_mma, phase);
         phase ^= 1u;
     }
@@ -687,6 +709,23 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             __half* bb = reinterpret_cast<__half*>(blk + tc::kOffB) + (size_t)(c0 / NS) * D * NS;
 #pragma unroll
             for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(bb + tc::sw_half(cc, g8)) = tc::f_to_h8(x + g8);
+        }
+    }
+    if (ok) {   // PU' (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (fp16 sw rows per 32-column slice)
+        const int q = warp & 3, chh = warp >> 2;
+        const uint32_t lb = (uint32_t)(32 * q) << 16;
+#pragma unroll 1
+        for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
+            float x[32];
+            tmem_ld32(t0 + lb + 128 + c0, x);
+            if (lane < 16) {
+                const int r = 16 * q + lane;
+                __half* pu = reinterpret_cast<__half*>(blk + tc::kOffPU) + (size_t)(c0 / NS) * C * NS;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) vmax = fmax_nan(vmax, fabsf(x[e]));
+#pragma unroll
+                for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::sw_half(r, g8)) = tc::f_to_h8(x + g8);
+            }
         }
     }
     if (tid < D) reinterpret_cast<float*>(blk + tc::kOffGC)[tid] = tgam[tid];

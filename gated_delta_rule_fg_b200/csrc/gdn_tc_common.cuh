@@ -21,7 +21,7 @@ constexpr float kMaxHalfSpan = 6.0f;
 // stored in the order g ^ ((x >> 1) & 3), so eight consecutive rows read as 16-byte
 // vectors hit eight different bank groups.
 constexpr uint32_t kOffN = 0;            // N = -K'^T W, fp16 128x128, K-major (m=i, k=c): SBO 2048, LBO 128
-constexpr uint32_t kOffQe = 32768;       // Qe fp16 64x128, MN-major (m=r, k=c): SBO 2048, LBO 128
+constexpr uint32_t kOffQe = 32768;       // Qe fp16 64x128 (m=r, k=c), SBO 2048, LBO 128: MN-major from intra_tc_kernel, K-major from the TMA-fed intra kernel
 constexpr uint32_t kOffB = 49152;        // b = K'^T U', fp16 [J][128][NS] (sw rows)
 constexpr uint32_t kOffPU = 81920;       // PU', fp16 [J][64][NS] (sw rows)
 constexpr uint32_t kOffGC = 98304;       // e^{g_last}, fp32 [128]

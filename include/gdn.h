@@ -58,9 +58,13 @@
  *     ran out) are recorded in the workspace and read with
  *     gdn_workspace_status().
  *   - The tensor-core path rounds its operands to fp16 (largest finite value
- *     65504).  The kernels do not check that range: a state whose entries
- *     exceed it (for instance from an S0 that large) gives undefined numbers,
- *     as out-of-range alpha and beta do.
+ *     65504).  Normalised q and k and the decay factors are always inside that
+ *     range; the value operand sqrt(beta) v, the per-chunk quantities that scale
+ *     with v and the fp16 copy of the state are checked, and a call whose values
+ *     (or state, for instance from an S0 that large) leave the range, or turn
+ *     NaN, records GDN_ERR_RANGE in the workspace status word (read with
+ *     gdn_workspace_status): its results are then not valid.  (gdn2_chunk_fwd
+ *     checks the state copy only.)  Out-of-range alpha and beta are not detected.
  */
 #ifndef GDN_B200_H
 #define GDN_B200_H
@@ -79,7 +83,7 @@ typedef enum {
     GDN_ERR_CUDA = 3,          /* a CUDA launch or copy failed (cudaGetLastError is left set) */
     GDN_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out; outputs are not valid */
     GDN_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or smaller than required */
-    GDN_ERR_RANGE = 6          /* reserved: the present kernels do not test the fp16 operand range */
+    GDN_ERR_RANGE = 6          /* device side: a value left the fp16 operand range of the tensor-core path */
 } gdn_status_t;
 
 typedef enum {
@@ -299,7 +303,15 @@ gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
 
 /* Waits for `stream`, then returns (and clears) the first device-side error
  * recorded in `workspace` by earlier calls: GDN_OK, GDN_ERR_TIMEOUT or
- * GDN_ERR_RANGE; GDN_ERR_CUDA if the wait itself failed. */
+ * GDN_ERR_RANGE; GDN_ERR_CUDA if the wait itself failed.
+ *
+ * Every device-side wait of the library is bounded (2 s); a wait that runs out
+ * records GDN_ERR_TIMEOUT and the kernel unwinds (its copies land, its tensor
+ * memory is released), leaving the context usable.  Test knob, unset in normal
+ * use: with the environment variable GDN_TEST_SCAN_SKIP_CHUNK=<c> set when a
+ * forward call is made, the tensor-core scan (bf16, d = 128, chunk 64) leaves
+ * chunk c unloaded and bounds its waits by 1 ms, so that call ends with
+ * GDN_ERR_TIMEOUT (and invalid outputs). */
 gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream);
 
 /* Static description of a status code. */

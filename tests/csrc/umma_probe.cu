@@ -244,3 +244,77 @@ extern "C" int umma_probe_sw(const void* A, const void* B, float* D, int M, int 
                                       K, a_mn, b_mn, err);
     return cudaGetLastError() == cudaSuccess ? 0 : 2;
 }
+
+// A operand copied from shared memory into tensor memory with tcgen05.cp (shape 128x256b: 128
+// lanes x 8 columns, i.e. one K step of 16 fp16 for 128 rows), from the K-major canonical
+// layout (8-row x 16-byte core matrices, LBO between K groups, SBO between row groups), then
+// the product with A from tensor memory.  Rows m >= M of the copied tile are padding.
+__global__ void probe_cp_kernel(const __half* A, const __half* B, float* D, int M, int N, int K, int b_mn,
+                                int* err) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tbase;
+    unsigned char* sA = sm;                 // 128 rows x K, K-major, LBO 128, SBO (K / 8) * 128
+    unsigned char* sB = sm + 128 * 128 * 2;
+    const uint32_t lbo_a = 128, sbo_a = (uint32_t)(K / 8) * 128;
+    uint32_t lbo_b, sbo_b;
+    strides(N, K, 0, lbo_b, sbo_b);
+    for (int idx = threadIdx.x; idx < 128 * K; idx += blockDim.x) {
+        const int m = idx / K, k = idx % K;
+        *reinterpret_cast<__half*>(sA + off_kmajor(m, k, sbo_a, lbo_a)) = m < M ? A[m * K + k] : __float2half(0.f);
+    }
+    for (int idx = threadIdx.x; idx < K * N; idx += blockDim.x) {
+        const int k = idx / N, n = idx % N;
+        uint32_t off = b_mn ? off_mnmajor(n, k, sbo_b, lbo_b) : off_kmajor(n, k, sbo_b, lbo_b);
+        *reinterpret_cast<__half*>(sB + off) = B[idx];
+    }
+    fence_async_smem();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+    if (warp == 0) { tmem_alloc(&tbase, 512); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t t0 = tbase;
+    const uint32_t tA = t0 + 256;
+    if (threadIdx.x == 0) {
+        for (int kk = 0; kk < K / 16; ++kk) {
+            const uint64_t s = sdesc(smem_u32(sA) + kk * 2 * lbo_a, lbo_a, sbo_a);
+            asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(tA + 8u * kk), "l"(s) : "memory");
+        }
+        const uint32_t id = idesc_f16(M == 64 ? 128 : M, N, false, b_mn, false);
+        for (int kk = 0; kk < K / 16; ++kk) {
+            const uint64_t b = sdesc(smem_u32(sB) + kk * 2 * lbo_b, lbo_b, sbo_b);
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(t0),
+                "r"(tA + 8u * kk), "l"(b), "r"((uint32_t)(kk > 0)), "r"(id)
+                : "memory");
+        }
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    if (!ok && lane == 0) atomicExch(err, 4);
+    tc_fence_after();
+    if (ok) {
+        for (int c0 = 0; c0 < N; c0 += 32) {
+            float v[32];
+            tmem_ld32(t0 + ((uint32_t)(32 * warp) << 16) + c0, v);
+            const int row = 32 * warp + lane;       // an M = 128 product: row m in lane m
+            if (row < M)
+                for (int j = 0; j < 32 && c0 + j < N; ++j) D[row * N + c0 + j] = v[j];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(t0, 512);
+}
+
+extern "C" int umma_probe_cp(const void* A, const void* B, float* D, int M, int N, int K, int b_mn, int* err) {
+    if ((M != 64 && M != 128) || N % 32 || N > 256 || K % 16 || K > 128) return 1;
+    size_t smem = 200 * 1024;
+    cudaFuncSetAttribute(probe_cp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    probe_cp_kernel<<<1, 128, smem>>>(static_cast<const __half*>(A), static_cast<const __half*>(B), D, M, N, K,
+                                      b_mn, err);
+    return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}

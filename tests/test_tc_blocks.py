@@ -2,7 +2,8 @@
 writes into the workspace (N = -K'^T W, Qe, b = K'^T U', PU', e^{g_last}) and compare them with the
 same quantities formed in fp64 numpy from their definitions (chunk-local cumulative
 log-decay g, A and P with the decay taken element by element, T = (I + A)^{-1}).
-The block layout is the library's internal contract between its two kernels."""
+The block layout is the library's internal contract between its two kernels (Qe is stored
+K-major, rows of 128 channels, for the scan's tensor-memory copy)."""
 import numpy as np
 import pytest
 
@@ -35,7 +36,7 @@ def decode(blk):
     i2, c2 = np.meshgrid(np.arange(128), np.arange(128), indexing="ij")
     N = h[(OFF_N + off_k(i2, c2, 2048, 128)) // 2].astype(np.float64)
     r2, c3 = np.meshgrid(np.arange(64), np.arange(128), indexing="ij")
-    Qe = h[(OFF_QE + off_mn(r2, c3, 2048, 128)) // 2].astype(np.float64)
+    Qe = h[(OFF_QE + off_k(r2, c3, 2048, 128)) // 2].astype(np.float64)
     jj = np.arange(128)
     bi, bj = np.meshgrid(np.arange(128), jj, indexing="ij")
     b = h[OFF_B // 2 + (bj // NS) * 128 * NS + sw(bi, bj % NS)].astype(np.float64)
