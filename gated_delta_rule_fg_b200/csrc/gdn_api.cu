@@ -5,6 +5,7 @@
 
 #include "gdn.h"
 #include "gdn_common.cuh"
+#include "gdn_nvtx.h"
 
 namespace gdn {
 // gdn_simt.cu
@@ -155,6 +156,7 @@ gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,
                            gdn_dtype_t dtype, unsigned flags,
                            void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_chunk_fwd");
     Problem p;
     gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false);
     if (st != GDN_OK) return st;
@@ -184,6 +186,7 @@ gdn_status_t gdn_plus_chunk_fwd(const void* q, const void* k, const void* v,
                                 gdn_dtype_t dtype, unsigned flags,
                                 void* workspace, size_t workspace_bytes,
                                 cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_plus_chunk_fwd");
     Problem p;
     gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, true);
     if (st != GDN_OK) return st;
@@ -207,6 +210,7 @@ gdn_status_t gdn_deltaproduct_fwd(const void* q, const void* k, const void* v,
                                   gdn_dtype_t dtype,
                                   void* workspace, size_t workspace_bytes,
                                   cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_deltaproduct_fwd");
     Problem p;
     gdn_status_t st = make_problem(p, B, H, T, n_h, dk, dv, chunk, dtype, 0u, true);
     if (st != GDN_OK) return st;
@@ -240,6 +244,7 @@ gdn_status_t gdn2_chunk_fwd(const void* q, const void* k, const void* v, const f
                             float* S_final, int B, int H, int T, int dk, int dv, int chunk,
                             gdn_dtype_t dtype, unsigned flags, int mode,
                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn2_chunk_fwd");
     Problem p;
     if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_SINGLE_STREAM)) return GDN_ERR_INVALID_ARG;
     if (mode < 0 || mode > 2) return GDN_ERR_INVALID_ARG;
@@ -291,6 +296,7 @@ gdn_status_t gdn_chunk_bwd(const void* q, const void* k, const void* v,
                            int B, int H, int T, int dk, int dv, int chunk,
                            gdn_dtype_t dtype, unsigned flags,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_chunk_bwd");
     Problem p;
     gdn_status_t st = make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false, beta_v != nullptr);
     if (st != GDN_OK) return st;
@@ -320,6 +326,7 @@ gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
                                 const float* S_in, float* S_out, void* out,
                                 int B, int H, int dk, int dv, gdn_dtype_t dtype, unsigned flags,
                                 cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_recurrent_step");
     if (B < 0 || H < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR)) return GDN_ERR_INVALID_ARG;
@@ -347,6 +354,7 @@ gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
 }
 
 gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream) {
+    NvtxRange nvtx_range("gdn_workspace_status");
     if (!workspace) return GDN_ERR_WORKSPACE;
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GDN_ERR_CUDA;
     int word = 0;

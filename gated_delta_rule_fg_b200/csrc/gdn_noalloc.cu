@@ -29,6 +29,7 @@
 #include <cuda.h>
 
 #include "gdn.h"
+#include "gdn_nvtx.h"
 
 namespace gdn {
 gdn_status_t chunk_fwd_check_args(const void* q, const void* k, const void* v, const float* alpha,
@@ -101,6 +102,7 @@ extern "C" gdn_status_t gdn_chunk_fwd_noalloc(const void* q, const void* k, cons
                                               int B, int H, int T, int dk, int dv, int chunk,
                                               gdn_dtype_t dtype, unsigned flags,
                                               cudaStream_t stream) {
+    gdn::NvtxRange nvtx_range("gdn_chunk_fwd_noalloc");
     // validation first: nothing is enqueued for a call that is rejected
     const gdn_status_t chk = gdn::chunk_fwd_check_args(q, k, v, alpha, beta, S0, out, S_final, B, H, T,
                                                        dk, dv, chunk, dtype, flags);

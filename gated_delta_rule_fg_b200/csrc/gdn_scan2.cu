@@ -3,7 +3,7 @@
 // the chunks of its range, one CTA per SM.  W = 2 carries a head on two SMs: the chain product
 // costs about the same for 64 columns as for 32, and the SMs it does not hold run intra CTAs.
 //
-// Per chunk c, with S_c in fp32 registers (row i per thread) and its fp16 copy in Sop[c % 3]:
+// Per chunk c, with S_c in fp32 registers (row i per thread) and its fp16 copy in Sop[c % kSl]:
 //   MMA_S: D_S = N_c S_c            -> S_{c+1} = Diag(gC) S_c + D_S + b_c   (the serial chain)
 //   MMA_O: D_O = [Qe_c; *] S_c      -> O_c = D_O + PU'_c                      (off the chain)
 // Both products take their A operand from tensor memory: four feeder warps copy N_c (128 rows)
@@ -15,9 +15,10 @@
 //
 // Warps: 0 .. 4W-1 state (lane quarter w % 4, slice w / 4), 4W .. 4W+3 N feeders (lane quarter
 // w - 4W), 4W+4 producer (bulk copies into three rings: {N, Qe}, {b slices, gC}, {PU' slices}),
-// 4W+5 MMA issuer, 4W+6 and 4W+7 Qe feeders and output writers (lane quarters 2 and 3: Qe rows
-// 0 .. 63 and D_O rows 64 .. 127).  Every hand-off is an mbarrier with a bounded wait; a wait that
-// runs out records GDN_ERR_TIMEOUT and the role unwinds.
+// 4W+5 chain MMA issuer, 4W+6 and 4W+7 Qe feeders (lane quarters 2 and 3: Qe
+// rows 0 .. 63 into lanes 64 .. 127), 4W+8 output MMA issuer, 4W+10 and 4W+11 output writers
+// (D_O lanes 64 .. 127; warp 4W+9 only fills the lane-quarter pattern).  Every hand-off is an
+// mbarrier with a bounded wait; a wait that runs out records GDN_ERR_TIMEOUT and the role unwinds.
 #include "gdn_tc_common.cuh"
 
 namespace gdn {
@@ -30,7 +31,7 @@ using tc::NS;
 template <int W>
 struct Cfg {
     static constexpr int NSW = NS * W;                       // columns of this CTA
-    static constexpr int kThreads = 32 * (4 * W + 8);
+    static constexpr int kThreads = 32 * (4 * W + 12);
     // Three rings, each released by the role that reads it last: {N, Qe} by the feeders once
     // copied into tensor memory, {b slices, gC} by the state warps, {PU' slices} by the output
     // warps (which run two chunks behind the chain, so their data must not hold back the state
@@ -42,11 +43,14 @@ struct Cfg {
     static constexpr uint32_t kBGBytes = 8192 * W + 512;     // b slices (fp16 sw rows), gC
     static constexpr uint32_t kPUBytes = 4096 * W;           // PU' slices (fp16 sw rows)
     static constexpr uint32_t kSopBytes = 8192 * W;          // S fp16 (k = i, n = j) MN-major SBO 2048 LBO 128
+    // Sop slots: S_c lives in slot c % kSl until MMA_S(c) and MMA_O(c) have read it; the output
+    // product may lag the chain by kSl - 2 chunks before the state warps wait for it
+    static constexpr int kSl = W == 1 ? 4 : 3;
     static constexpr uint32_t kRingNQ = 0;
     static constexpr uint32_t kRingBG = kRingNQ + kNQ * kNQBytes;
     static constexpr uint32_t kRingPU = kRingBG + kBG * kBGBytes;
     static constexpr uint32_t kSop = kRingPU + kPU * kPUBytes;
-    static constexpr uint32_t kBar = kSop + 3 * kSopBytes;
+    static constexpr uint32_t kBar = kSop + kSl * kSopBytes;
     static constexpr uint32_t kTslot = kBar + 512;
     static constexpr uint32_t kSmem = kTslot + 64;
     // tensor memory columns (512 allocated): D_S, D_O[2], Qe[2] (64 each), N[2] (64 each)
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
     constexpr uint32_t kRingNQ = K::kRingNQ, kRingBG = K::kRingBG, kRingPU = K::kRingPU, kSop = K::kSop;
     constexpr uint32_t kSopBytes = K::kSopBytes, kBar = K::kBar, kTslot = K::kTslot;
     constexpr uint32_t kTS = K::kTS, kTO = K::kTO, kTQ = K::kTQ, kTN = K::kTN;
-    constexpr int kNO = K::kNO;
+    constexpr int kNO = K::kNO, kSl = K::kSl;
     extern __shared__ __align__(1024) uint8_t sm[];
     const int slice0 = blockIdx.x * W;                     // first 32-column slice of this CTA
     const int bh = blockIdx.y;
@@ -118,7 +122,9 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
     uint64_t* q_free = q_ready + kNO;      // [kNO] MMA_O that read Qe buffer done
     uint64_t* bar_o = q_free + kNO;        // [kNO] MMA_O done, per D_O buffer
     uint64_t* o_free = bar_o + kNO;        // [kNO] D_O buffer read (the 2 output warps)
-    uint64_t* bar_d = o_free + kNO;        // drain: the MMA thread's last products done
+    uint64_t* s_slot = o_free + kNO;       // [kSl] S_c written into Sop slot c % kSl (4W state warps)
+    uint64_t* o_done = s_slot + kSl;       // [kSl] MMA_O that read Sop slot c % kSl done
+    uint64_t* bar_d = o_done + kSl;        // drain: both MMA threads' last products done
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kTslot);
     const uint8_t* blocks = static_cast<const uint8_t*>(p.inter) + (size_t)bh * p.NC * tc::kBlockBytes;
     const int nloc = ce - cb;
@@ -143,7 +149,11 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             mbar_init(&bar_o[i], 1);
             mbar_init(&o_free[i], 2);
         }
-        mbar_init(bar_d, 1);
+        for (int i = 0; i < kSl; ++i) {
+            mbar_init(&s_slot[i], 4 * W);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(bar_d, 2);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -208,39 +218,47 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
                 if (ld_pu[i] >= 0) mbar_wait(&fullPU[i], (ld_pu[i] / kPU) & 1, lim);
         }
     } else if (warp == 4 * W + 5) {
-        // ------------------------------------------------------------ MMA issuer (one thread)
+        // ------------------------------------------------------------ chain MMA issuer (one thread)
+        // A thread that issues tcgen05.mma is held for about the time the tensor pipe takes to
+        // accept each instruction, while two issuing threads proceed side by side; so the chain
+        // product has a thread of its own, and the output products another (warp 4W+8).
         if (lane == 0) {
             const uint32_t idS = idesc_f16(128, NSW, false, true);
-            const uint32_t idO = idesc_f16(128, NSW, false, true);
-            auto issue_o = [&](int cc) -> bool {
-                const int bo = cc % kNO, uo = cc / kNO;        // buffer, and its use count
-                if (!mbar_wait(&q_ready[bo], uo & 1, lim)) return false;
-                if (uo >= 1 && !mbar_wait(&o_free[bo], (uo - 1) & 1, lim)) return false;
+            for (int ch = 0; ch < nloc && ok; ++ch) {
+                if (!mbar_wait(s_ready, ch & 1, lim) || !mbar_wait(&n_ready[ch & 1], (ch >> 1) & 1, lim)) { ok = false; break; }
                 tc_fence_after();
-                const uint64_t b0 = sdesc(smem_u32(sm + kSop + (cc % 3) * kSopBytes), 128, 2048);
+                const uint64_t b0 = sdesc(smem_u32(sm + kSop + (ch % kSl) * kSopBytes), 128, 2048);
+                const uint32_t an = t0 + kTN + 64u * (ch & 1);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) mma_ta(t0 + kTS, an + 8u * kk, b0 + 16 * kk, idS, kk > 0);
+                mma_commit(bar_s);
+                mma_commit(&n_free[ch & 1]);
+            }
+            if (!ok) tc::record_timeout(p.status);
+            // drain: every product this thread issued has completed before the tensor memory goes
+            mma_commit(bar_d);
+            if (!mbar_wait(bar_d, 0, lim)) tc::record_timeout(p.status);
+        }
+    } else if (warp == 4 * W + 8) {
+        // ------------------------------------------------------------ output MMA issuer (one thread)
+        // MMA_O(c) reads S_c from Sop slot c % kSl once the state warps have written it; its
+        // completion (o_done) lets them write S_{c+kSl} there.
+        if (lane == 0) {
+            const uint32_t idO = idesc_f16(128, NSW, false, true);
+            for (int cc = 0; cc < nloc && ok; ++cc) {
+                const int bo = cc % kNO, uo = cc / kNO;        // buffer, and its use count
+                if (!mbar_wait(&s_slot[cc % kSl], (cc / kSl) & 1, lim) || !mbar_wait(&q_ready[bo], uo & 1, lim) ||
+                    (uo >= 1 && !mbar_wait(&o_free[bo], (uo - 1) & 1, lim))) { ok = false; break; }
+                tc_fence_after();
+                const uint64_t b0 = sdesc(smem_u32(sm + kSop + (cc % kSl) * kSopBytes), 128, 2048);
                 const uint32_t aq = t0 + kTQ + 64u * bo;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) mma_ta(t0 + kTO + NSW * bo, aq + 8u * kk, b0 + 16 * kk, idO, kk > 0);
                 mma_commit(&bar_o[bo]);
                 mma_commit(&q_free[bo]);
-                return true;
-            };
-            for (int ch = 0; ch < nloc && ok; ++ch) {
-                if (!mbar_wait(s_ready, ch & 1, lim) || !mbar_wait(&n_ready[ch & 1], (ch >> 1) & 1, lim)) { ok = false; break; }
-                tc_fence_after();
-                {
-                    const uint64_t b0 = sdesc(smem_u32(sm + kSop + (ch % 3) * kSopBytes), 128, 2048);
-                    const uint32_t an = t0 + kTN + 64u * (ch & 1);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) mma_ta(t0 + kTS, an + 8u * kk, b0 + 16 * kk, idS, kk > 0);
-                    mma_commit(bar_s);
-                    mma_commit(&n_free[ch & 1]);
-                }
-                if (ch > 0 && !issue_o(ch - 1)) { ok = false; break; }
+                mma_commit(&o_done[cc % kSl]);
             }
-            if (ok && nloc > 0) ok = issue_o(nloc - 1);
             if (!ok) tc::record_timeout(p.status);
-            // drain: every product this thread issued has completed before the tensor memory goes
             mma_commit(bar_d);
             if (!mbar_wait(bar_d, 0, lim)) tc::record_timeout(p.status);
         }
@@ -260,7 +278,10 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
         for (int j = 0; j < NS; j += 8) tc::st16(sm + kSop, off_mnmajor(NS * sl + j, row, 2048, 128), tc::f_to_h8(S + j));
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_ready);
+        if (lane == 0) {
+            mbar_arrive(s_ready);
+            mbar_arrive(&s_slot[0]);
+        }
         for (int ch = 0; ch < nloc && ok; ++ch) {
             const int sb = ch % kBG;
             const uint8_t* bp = sm + kRingBG + sb * kBGBytes;
@@ -279,13 +300,21 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
                 }
             }
             const float gc = reinterpret_cast<const float*>(bp + 8192 * W)[row];
+            // Sop slot (ch + 1) % kSl last held S_{ch+1-kSl}: its output product must be done before
+            // S_{ch+1} goes there (its chain product is: MMA_S(ch) completes after it).  Checked
+            // before the chain product's wait, off the chain's path.
+            if (ch + 1 >= kSl &&
+                !__all_sync(0xffffffffu, mbar_wait(&o_done[(ch + 1) % kSl], ((ch + 1 - kSl) / kSl) & 1, lim))) {
+                ok = false;
+                break;
+            }
             if (!__all_sync(0xffffffffu, mbar_wait(bar_s, ch & 1, lim))) { ok = false; break; }
             tc_fence_after();
             float d[NS];
             tmem_ld32(t0 + kTS + lanebase + NS * sl, d);
 #pragma unroll
             for (int j = 0; j < NS; ++j) S[j] = fmaf(gc, S[j], d[j] + bv[j]);
-            uint8_t* snext = sm + kSop + ((ch + 1) % 3) * kSopBytes;
+            uint8_t* snext = sm + kSop + ((ch + 1) % kSl) * kSopBytes;
 #pragma unroll
             for (int j = 0; j < NS; j += 8) tc::st16(snext, off_mnmajor(NS * sl + j, row, 2048, 128), tc::f_to_h8(S + j));
             fence_async_smem();
@@ -293,6 +322,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(s_ready);                          // this warp's part of S_{ch+1} is in Sop
+                mbar_arrive(&s_slot[(ch + 1) % kSl]);
                 mbar_arrive(&emptyBG[sb]);
             }
 #pragma unroll
@@ -327,69 +357,71 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             }
         }
         if (!ok && lane == 0) tc::record_timeout(p.status);
-    } else if (warp >= 4 * W + 6) {
-        // ------------------------------------------------------------ Qe feeders / outputs (warps 4W+6, 4W+7)
+    } else if (warp < 4 * W + 8) {
+        // ------------------------------------------------------------ Qe feeders (warps 4W+6, 4W+7)
         const int q = warp & 3;                                // TMEM lane quarter: 2 or 3
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-        const int row = 32 * (q - 2) + lane;                   // Qe row / output row of the chunk
+        const int row = 32 * (q - 2) + lane;                   // Qe row of the chunk
+        // Qe_it into buffer it % kNO (lanes 64 .. 127) once MMA_O(it - kNO) has read it
+        for (int it = 0; it < nloc && ok; ++it) {
+            const int s2 = it % kNQ;
+            bool got = mbar_wait(&fullNQ[s2], (it / kNQ) & 1, lim);
+            const int bq = it % kNO, uq = it / kNO;
+            if (uq >= 1) got = got && mbar_wait(&q_free[bq], (uq - 1) & 1, lim);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            rows_to_tmem(sm + kRingNQ + s2 * kNQBytes + 32768, row, t0 + kTQ + 64u * bq + lanebase);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&q_ready[bq]);
+                mbar_arrive(&emptyNQ[s2]);
+            }
+        }
+        if (!ok && lane == 0) tc::record_timeout(p.status);
+    } else if (warp >= 4 * W + 10) {
+        // ------------------------------------------------------------ outputs (warps 4W+10, 4W+11)
+        const int q = warp & 3;                                // TMEM lane quarter: 2 or 3
+        const uint32_t lanebase = (uint32_t)(32 * q) << 16;
+        const int row = 32 * (q - 2) + lane;                   // output row of the chunk (D_O lane 64 + row)
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-        // iteration it: Qe_it into buffer it % kNO (lanes 64 .. 127) once MMA_O(it - kNO) has read
-        // it, then the outputs of chunk it - 2
-        for (int it = 0; it < nloc + 2 && ok; ++it) {
-            if (it < nloc) {
-                const int s2 = it % kNQ;
-                bool got = mbar_wait(&fullNQ[s2], (it / kNQ) & 1, lim);
-                const int bq = it % kNO, uq = it / kNO;
-                if (uq >= 1) got = got && mbar_wait(&q_free[bq], (uq - 1) & 1, lim);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                tc_fence_after();
-                rows_to_tmem(sm + kRingNQ + s2 * kNQBytes + 32768, row, t0 + kTQ + 64u * bq + lanebase);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&q_ready[bq]);
-                    mbar_arrive(&emptyNQ[s2]);
-                }
-            }
-            const int oc = it - 2;
-            if (oc >= 0) {
-                const int sp = oc % kPU;
-                const int bo = oc % kNO;
-                const bool got = mbar_wait(&fullPU[sp], (oc / kPU) & 1, lim) && mbar_wait(&bar_o[bo], (oc / kNO) & 1, lim);
-                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                tc_fence_after();
-                const int s = (cb + oc) * C + row;
-                RowRef ro{};
-                const bool write = s < p.L && (ro = row_ref(p, b, h, s)).has_q;
+        for (int oc = 0; oc < nloc && ok; ++oc) {
+            const int sp = oc % kPU;
+            const int bo = oc % kNO;
+            const bool got = mbar_wait(&fullPU[sp], (oc / kPU) & 1, lim) && mbar_wait(&bar_o[bo], (oc / kNO) & 1, lim);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            const int s = (cb + oc) * C + row;
+            RowRef ro{};
+            const bool write = s < p.L && (ro = row_ref(p, b, h, s)).has_q;
 #pragma unroll 1
-                for (int sl = 0; sl < W; ++sl) {
-                    float d[NS];
-                    tmem_ld32(t0 + kTO + NSW * bo + NS * sl + lanebase, d);
-                    if (sl == W - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&o_free[bo]);
-                    }
-                    if (write) {
-                        const __half* pu = reinterpret_cast<const __half*>(sm + kRingPU + sp * kPUBytes) + sl * (C * NS);
-                        uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + (slice0 + sl) * NS);
+            for (int sl = 0; sl < W; ++sl) {
+                float d[NS];
+                tmem_ld32(t0 + kTO + NSW * bo + NS * sl + lanebase, d);
+                if (sl == W - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&o_free[bo]);
+                }
+                if (write) {
+                    const __half* pu = reinterpret_cast<const __half*>(sm + kRingPU + sp * kPUBytes) + sl * (C * NS);
+                    uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + (slice0 + sl) * NS);
 #pragma unroll
-                        for (int g8 = 0; g8 < NS; g8 += 8) {
-                            const uint4 pv = *reinterpret_cast<const uint4*>(pu + tc::sw_half(row, g8));
-                            const __half2* ph = reinterpret_cast<const __half2*>(&pv);
-                            __nv_bfloat162 o2[4];
+                    for (int g8 = 0; g8 < NS; g8 += 8) {
+                        const uint4 pv = *reinterpret_cast<const uint4*>(pu + tc::sw_half(row, g8));
+                        const __half2* ph = reinterpret_cast<const __half2*>(&pv);
+                        __nv_bfloat162 o2[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 pf = __half22float2(ph[e]);
-                                o2[e] = __floats2bfloat162_rn(pf.x + d[g8 + 2 * e], pf.y + d[g8 + 2 * e + 1]);
-                            }
-                            dst[g8 / 8] = *reinterpret_cast<uint4*>(o2);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 pf = __half22float2(ph[e]);
+                            o2[e] = __floats2bfloat162_rn(pf.x + d[g8 + 2 * e], pf.y + d[g8 + 2 * e + 1]);
                         }
+                        dst[g8 / 8] = *reinterpret_cast<uint4*>(o2);
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&emptyPU[sp]);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&emptyPU[sp]);
         }
         if (!ok && lane == 0) tc::record_timeout(p.status);
     }

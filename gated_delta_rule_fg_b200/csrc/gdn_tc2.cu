@@ -80,6 +80,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kBarOff);
     uint64_t* bar_mma = bar_tma + 1;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kBarOff + 16);
+    // Every round of products is issued by two threads in different warps (thread 0 and thread 32),
+    // each committing to its own barrier: a thread issuing tcgen05.mma is held for about the time
+    // the tensor pipe takes to accept each instruction, and two issuers proceed side by side.
+    uint64_t* bar_mma2 = reinterpret_cast<uint64_t*>(sm + kBarOff + 24);
     float* scr = reinterpret_cast<float*>(sm + kScr);
     float* tgam = reinterpret_cast<float*>(sm + kTab);
     float* tref = tgam + 128;
@@ -95,6 +99,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_mma2, 1);
         fence_mbar_init();
         if (kDP) {
             const int t0 = s0 / p.nh;
@@ -370,18 +375,21 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 
     // ---------------------------------------------------------------- [A; P] = [KG; QG] KI^T
     if (!fallback) {
-        if (tid == 0 && ok) {
+        // channels 0-63 (thread 0) into columns 0-63, channels 64-127 (thread 32) into 64-127;
+        // the epilogue adds the two
+        if ((tid == 0 || tid == 32) && ok) {
             const uint32_t id = idesc_f16(128, 64, false, false);
+            const int hk = tid >> 5;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (uint32_t)((kk >> 2) * 16384 + (kk & 3) * 32);
-                const uint32_t kioff = (uint32_t)((kk >> 2) * 8192 + (kk & 3) * 32);
-                mma_f16(t0, sdesc_sw128(base + kKQ + koff, 16, 1024), sdesc_sw128(base + kKI + kioff, 16, 1024), id,
-                        kk > 0);
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const uint32_t koff = (uint32_t)(hk * 16384 + k4 * 32);
+                const uint32_t kioff = (uint32_t)(hk * 8192 + k4 * 32);
+                mma_f16(t0 + 64u * hk, sdesc_sw128(base + kKQ + koff, 16, 1024), sdesc_sw128(base + kKI + kioff, 16, 1024),
+                        id, k4 > 0);
             }
-            mma_commit(bar_mma);
+            mma_commit(hk ? bar_mma2 : bar_mma);
         }
-        ok = ok && mbar_wait(bar_mma, phase);
+        ok = ok && mbar_wait(bar_mma, phase) && mbar_wait(bar_mma2, phase);
         phase ^= 1u;
     } else if (warp < 4) {
         // exact fp32 Gram products, element by element (decay formed per pair of rows)
@@ -413,6 +421,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
         const int q = warp & 3, chh = warp >> 2;
         float d[32];
         tmem_ld32(t0 + ((uint32_t)(32 * q) << 16) + 32 * chh, d);
+        if (!fallback) {
+            float d2[32];
+            tmem_ld32(t0 + ((uint32_t)(32 * q) << 16) + 64 + 32 * chh, d2);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) d[i] += d2[i];
+        }
         const int rho = 32 * q + lane;
         if (rho < 64) {
             const int rw = rho;
@@ -556,18 +570,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 
     // ---------------------------------------------------------------- Y = KI^T T, Z = P T
     if (ok) {
-        if (tid == 0) {
+        if (tid == 0) {               // Y
             const uint32_t idY = idesc_f16(128, 64, true, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(t0 + 64, sdesc_sw128(base + kKI + kk * 2048, 8192, 1024), sdesc(base + kT16 + kk * 2048, 1024, 128),
+                        idY, kk > 0);
+            mma_commit(bar_mma);
+        } else if (tid == 32) {       // Z
             const uint32_t idZ = idesc_f16(64, 64, false, true);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bT = sdesc(base + kT16 + kk * 2048, 1024, 128);
-                mma_f16(t0 + 64, sdesc_sw128(base + kKI + kk * 2048, 8192, 1024), bT, idY, kk > 0);
-                mma_f16(t0 + 128, sdesc(base + kP16 + kk * 256, 128, 1024), bT, idZ, kk > 0);
-            }
-            mma_commit(bar_mma);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(t0 + 128, sdesc(base + kP16 + kk * 256, 128, 1024), sdesc(base + kT16 + kk * 2048, 1024, 128),
+                        idZ, kk > 0);
+            mma_commit(bar_mma2);
         }
-        ok = mbar_wait(bar_mma, phase);
+        ok = mbar_wait(bar_mma, phase) && mbar_wait(bar_mma2, phase);
         phase ^= 1u;
     }
     ok = __syncthreads_and(ok);
@@ -593,13 +611,6 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             }
         }
     }
-    for (int idx = tid; idx < 512; idx += NT) {   // identity in Z's layout, over P16
-        const int ri = idx & 63, j = idx >> 6;
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = (8 * j + e == ri) ? 1.f : 0.f;
-        tc::st16(sm + kP16, off_kmajor(ri, 8 * j, 1024, 128), tc::f_to_h8(f));
-    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -607,25 +618,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 
     // ---------------------------------------------------------------- N~ = Y KG, Qe~ = QG - Z KG
     if (ok) {
-        if (tid == 0) {
+        if (tid == 0) {               // N~ = Y KG
             const uint32_t idN = idesc_f16(128, 128, false, true);
-            const uint32_t idQ = idesc_f16(64, 128, false, true);
-            const uint32_t idQn = idesc_f16(64, 128, false, true, true);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bKG = sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024);
-                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), bKG, idN, kk > 0);
-                // Qe~ = I QG - Z KG (M = 64: the identity, then Z, as A; QG and KG as MN-major B)
-                mma_f16(t0 + 128, sdesc(base + kP16 + kk * 256, 128, 1024),
-                        sdesc_sw128(base + kKQ + 8192 + kk * 2048, 16384, 1024), idQ, kk > 0);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024),
+                        idN, kk > 0);
+            mma_commit(bar_mma);
+        } else if (tid == 32) {       // -Z KG (M = 64; the epilogue adds QG)
+            const uint32_t idQn = idesc_f16(64, 128, false, true, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024),
-                        idQn, true);
-            mma_commit(bar_mma);
+                        idQn, kk > 0);
+            mma_commit(bar_mma2);
         }
-        ok = mbar_wait(bar_mma, phase);
+        ok = mbar_wait(bar_mma, phase) && mbar_wait(bar_mma2, phase);
         phase ^= 1u;
     }
     ok = __syncthreads_and(ok);
@@ -651,14 +659,21 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
                     *reinterpret_cast<uint4*>(blk + tc::kOffN + off_kmajor(cc, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
             }
         }
-        // Qe = Qe~ diag(col) (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (K-major
-        // (m = r, k = c): SBO 2048, LBO 128)
+        // Qe = (QG - Z KG) diag(col) (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block
+        // (K-major (m = r, k = c): SBO 2048, LBO 128)
 #pragma unroll 1
         for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
             float x[32];
             tmem_ld32(t0 + lb + 128 + c0, x);
             if (lane < 16) {
                 const int r = 16 * q + lane;
+#pragma unroll
+                for (int g8 = 0; g8 < 32; g8 += 8) {
+                    float qg[8];
+                    tc::h8_to_f(*reinterpret_cast<const uint4*>(sm + kKQ + 8192 + sw128_off(r, c0 + g8, 16384)), qg);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[g8 + e] += qg[e];
+                }
 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 cs = *reinterpret_cast<const float4*>(tcol + c0 + e4);
@@ -675,18 +690,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     tc_fence_after();
     // ---------------------------------------------------------------- b~ = Y V, PU' = Z V
     if (ok) {
-        if (tid == 0) {
+        if (tid == 0) {               // b~ = Y V
             const uint32_t idN = idesc_f16(128, 128, false, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), sdesc_sw128(base + kV + kk * 2048, 8192, 1024),
+                        idN, kk > 0);
+            mma_commit(bar_mma);
+        } else if (tid == 32) {       // PU' = Z V
             const uint32_t idP = idesc_f16(64, 128, false, true);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bV = sdesc_sw128(base + kV + kk * 2048, 8192, 1024);
-                mma_f16(t0 + 0, sdesc(base + kA32 + kk * 256, 128, 1024), bV, idN, kk > 0);
-                mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), bV, idP, kk > 0);
-            }
-            mma_commit(bar_mma);
+            for (int kk = 0; kk < 4; ++kk)
+                mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), sdesc_sw128(base + kV + kk * 2048, 8192, 1024),
+                        idP, kk > 0);
+            mma_commit(bar_mma2);
         }
-        ok = mbar_wait(bar_mma, phase);
+        ok = mbar_wait(bar_mma, phase) && mbar_wait(bar_mma2, phase);
         phase ^= 1u;
     }
     ok = __syncthreads_and(ok);

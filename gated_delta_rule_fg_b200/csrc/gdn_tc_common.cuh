@@ -53,6 +53,16 @@ __device__ __forceinline__ void bf8_to_f(const uint4 u, float (&f)[8]) {
     }
 }
 
+__device__ __forceinline__ void h8_to_f(const uint4 u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
 __device__ __forceinline__ uint4 f_to_h8(const float* f) {
     uint4 u;
     __half2 h0 = __floats2half2_rn(f[0], f[1]);
