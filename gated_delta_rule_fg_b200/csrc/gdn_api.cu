@@ -46,7 +46,10 @@ gdn_status_t make_problem(Problem& p, int B, int H, int T, int nh, int dk, int d
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
     if (flags & ~(unsigned)(GDN_ALPHA_SCALAR | GDN_BETA_SCALAR | GDN_SINGLE_STREAM)) return GDN_ERR_INVALID_ARG;
     if (!dim_ok(dk) || !dim_ok(dv)) return GDN_ERR_UNSUPPORTED;
-    if (chunk != 16 && chunk != 32 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+    if (chunk != 16 && chunk != 32 && chunk != 64 && chunk != 128) return GDN_ERR_UNSUPPORTED;
+    // chunk 128 is evaluated as 64-row chunks: the chunk length changes only the order of the
+    // rounding, not what is computed, and the kernels tile at most 64 rows
+    if (chunk == 128) chunk = 64;
     if (dp && (nh < 1 || nh > 4)) return GDN_ERR_UNSUPPORTED;
     const bool beta_scalar = dp || (flags & GDN_BETA_SCALAR);
     if (!beta_scalar && !plus && dk != dv) return GDN_ERR_INVALID_ARG;   // sqrt(beta) scales v too

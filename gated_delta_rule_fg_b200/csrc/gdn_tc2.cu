@@ -21,8 +21,9 @@
 //   Qe = (QG - Z KG) diag(ref)            (=  Q^ e^g - P W)
 //   PU' = Z V
 // because K' = KI diag(ref) and W = T KG diag(ref).  Four rounds of tensor-core products:
-// [A; P]; Y and Z; N~ and Qe~; b~ and PU'.  Qe is stored K-major (rows of 128 channels), the
-// layout the scan copies into tensor memory as an A operand.
+// [A; P]; Y and Z; N~ = Y KG and -Z KG (the Qe epilogue adds QG from shared memory); b~ and
+// PU'.  Each round is issued by two threads (see bar_mma2).  Qe is stored K-major (rows of 128
+// channels), the layout the scan copies into tensor memory as an A operand.
 #include <cuda.h>
 
 #include "gdn_tc_common.cuh"
@@ -47,8 +48,7 @@ constexpr uint32_t kA32 = 65536;     // A, then T in place: fp32 64x64 (tc::sw64
                                      //   (K-major (m = channel, k = row): SBO 1024, LBO 128)
 constexpr uint32_t kT16 = 81920;     // T fp16 (k = row, n = column): MN-major SBO 128, LBO 1024;
                                      //   later Z fp16 (n = row r, k = r'): K-major SBO 1024, LBO 128
-constexpr uint32_t kP16 = 90112;     // P fp16 (m = row, k = column): K-major SBO 1024, LBO 128;
-                                     //   later the identity, in Z's layout
+constexpr uint32_t kP16 = 90112;     // P fp16 (m = row, k = column): K-major SBO 1024, LBO 128
 constexpr uint32_t kScr = 98304;     // 8 KB: row-group decay totals [16][128]; solve temporaries
 constexpr uint32_t kTab = 106496;    // fp32 [5][128]: gamma, ref, 1/ref, row scale, column scale
 constexpr uint32_t kBarOff = 109056; // mbarriers (TMA, MMA), TMEM base

@@ -110,8 +110,10 @@ size_t gdn_chunk_fwd_workspace_size(int B, int H, int T, int dk, int dv, int chu
  *   S0 (may be NULL), S_final (may be NULL): float32 [B,H,dk,dv].
  * Sizes: B, H, T >= 0 (zero is a no-op that still writes S_final = S0 or 0;
  * with T == 0 the token pointers may be NULL); dk, dv in {32, 64, 128};
- * chunk in {16, 32, 64}.  Channel-wise beta needs dk == dv (sqrt(beta) multiplies v).
- * T need not be a multiple of chunk.  GDN_BF16 with chunk == 64 and
+ * chunk in {16, 32, 64, 128}; chunk 128 is evaluated as 64-row chunks (the same
+ * recurrence, bit for bit the result of chunk 64: the kernels tile at most 64
+ * rows).  Channel-wise beta needs dk == dv (sqrt(beta) multiplies v).
+ * T need not be a multiple of chunk.  GDN_BF16 with chunk 64 (or 128) and
  * dk == dv == 128 runs on the tensor-core path; other GDN_BF16 shapes and all
  * GDN_F32 shapes run on the float32 CUDA-core path. */
 gdn_status_t gdn_chunk_fwd(const void* q, const void* k, const void* v,

@@ -80,7 +80,12 @@ def test_argument_validation_before_launch(L):
     assert _call(L, flags=8) == ops.GDN_ERR_INVALID_ARG
     assert _call(L, dk=64, dv=128) == ops.GDN_ERR_INVALID_ARG
     assert _call(L, dk=96, dv=96) == ops.GDN_ERR_UNSUPPORTED
-    assert _call(L, chunk=128) == ops.GDN_ERR_UNSUPPORTED
+    assert _call(L, chunk=256) == ops.GDN_ERR_UNSUPPORTED
+    # chunk 128 is accepted and evaluated as 64-row chunks: same workspace and launches as chunk 64
+    for dt, d in ((ops.GDN_BF16, 128), (ops.GDN_F32, 64)):
+        assert L.gdn_chunk_fwd_workspace_size(1, 4, 1000, d, d, 128, dt, 0) == \
+            L.gdn_chunk_fwd_workspace_size(1, 4, 1000, d, d, 64, dt, 0) > 0
+        assert L.gdn_chunk_fwd_launches(1, 4, 1000, d, d, 128, dt, 0) == L.gdn_chunk_fwd_launches(1, 4, 1000, d, d, 64, dt, 0)
     assert _call(L, chunk=0) == ops.GDN_ERR_UNSUPPORTED
     assert _call(L, ws=None) == ops.GDN_ERR_WORKSPACE
     assert _call(L, ws=FAKE + 16) == ops.GDN_ERR_WORKSPACE       # not 256-byte aligned

@@ -161,3 +161,19 @@ def test_single_stream_flag_same_result():
     o2, s2 = ops.chunk_fwd(*args, chunk=64, single_stream=True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
+@pytest.mark.parametrize("dtype,dk", [("bf16", 128), ("f32", 64)])
+def test_chunk_128_is_chunk_64(dtype, dk):
+    """chunk 128 is accepted and evaluated as 64-row chunks: bit for bit the chunk-64 result
+    (tensor-core path at bf16 d 128, float32 path at d 64), and within the tolerance of the
+    oracle's token-by-token recurrence."""
+    import oracle
+    cfg, x = _inputs(dtype, T=333, dk=dk)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    o64, s64 = _run(x, dtype, 64)
+    o128, s128 = _run(x, dtype, 128)
+    assert np.array_equal(o64, o128) and np.array_equal(s64, s128)
+    ro, rs = oracle.gdn_seq(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"])
+    parity(o128, ro, tol, out_bf16=dtype == "bf16")
+    parity(s128, rs, tol)
