@@ -40,8 +40,8 @@ struct Cfg {
     static constexpr int kBG = W == 1 ? 4 : 3;               // {b, gC} ring depth
     static constexpr int kPU = W == 1 ? 4 : 3;               // {PU'} ring depth
     static constexpr uint32_t kNQBytes = 32768 + 16384;      // N, then Qe (K-major, SBO 2048, LBO 128)
-    static constexpr uint32_t kBGBytes = 8192 * W + 512;     // b slices (fp16 sw rows), gC
-    static constexpr uint32_t kPUBytes = 4096 * W;           // PU' slices (fp16 sw rows)
+    static constexpr uint32_t kBGBytes = 8192 * W + 512;     // b slices (fp16 group-major), gC
+    static constexpr uint32_t kPUBytes = 4096 * W;           // PU' slices (fp16 group-major)
     static constexpr uint32_t kSopBytes = 8192 * W;          // S fp16 (k = i, n = j) MN-major SBO 2048 LBO 128
     // Sop slots: S_c lives in slot c % kSl until MMA_S(c) and MMA_O(c) have read it; the output
     // product may lag the chain by kSl - 2 chunks before the state warps wait for it
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             float bv[NS];
 #pragma unroll
             for (int g8 = 0; g8 < NS; g8 += 8) {
-                const uint4 v = *reinterpret_cast<const uint4*>(bsm + tc::sw_half(row, g8));
+                const uint4 v = *reinterpret_cast<const uint4*>(bsm + tc::grp_half(row, g8, D));
                 const __half2* hh = reinterpret_cast<const __half2*>(&v);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
                     uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + (slice0 + sl) * NS);
 #pragma unroll
                     for (int g8 = 0; g8 < NS; g8 += 8) {
-                        const uint4 pv = *reinterpret_cast<const uint4*>(pu + tc::sw_half(row, g8));
+                        const uint4 pv = *reinterpret_cast<const uint4*>(pu + tc::grp_half(row, g8, C));
                         const __half2* ph = reinterpret_cast<const __half2*>(&pv);
                         __nv_bfloat162 o2[4];
 #pragma unroll

@@ -92,10 +92,6 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     float* tcol = tgam + 512;
     float* A32 = reinterpret_cast<float*>(sm + kA32);
 
-    if (warp == 0) {
-        tmem_alloc(tslot, 256);
-        tmem_relinquish();
-    }
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
@@ -169,6 +165,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 #pragma unroll
             for (int e = 0; e < 8; ++e) be[i][e] = bb;
         }
+    }
+    // the tensor memory is taken once the q, k, v boxes and this warp's alpha / beta loads are in
+    // flight (its latency then overlaps theirs)
+    if (warp == 0) {
+        tmem_alloc(tslot, 256);
+        tmem_relinquish();
     }
     // cumulative product over this thread's four rows; the row-group total goes to scr
 #pragma unroll
@@ -711,7 +713,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     ok = __syncthreads_and(ok);
     if (!ok && tid == 0) tc::record_timeout(p.status);
     tc_fence_after();
-    if (ok) {                    // b = diag(row) b~ -> block (fp16 sw rows, one 32-column slice per load)
+    if (ok) {                    // b = diag(row) b~ -> block (fp16 group-major slices, one per load)
         const int q = warp & 3, chh = warp >> 2;
         const int cc = 32 * q + lane;
         const float rs = trow[cc];
@@ -727,10 +729,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             }
             __half* bb = reinterpret_cast<__half*>(blk + tc::kOffB) + (size_t)(c0 / NS) * D * NS;
 #pragma unroll
-            for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(bb + tc::sw_half(cc, g8)) = tc::f_to_h8(x + g8);
+            for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(bb + tc::grp_half(cc, g8, D)) = tc::f_to_h8(x + g8);
         }
     }
-    if (ok) {   // PU' (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (fp16 sw rows per 32-column slice)
+    if (ok) {   // PU' (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (fp16 group-major slices)
         const int q = warp & 3, chh = warp >> 2;
         const uint32_t lb = (uint32_t)(32 * q) << 16;
 #pragma unroll 1
@@ -743,7 +745,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 #pragma unroll
                 for (int e = 0; e < 32; ++e) vmax = fmax_nan(vmax, fabsf(x[e]));
 #pragma unroll
-                for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::sw_half(r, g8)) = tc::f_to_h8(x + g8);
+                for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::grp_half(r, g8, C)) = tc::f_to_h8(x + g8);
             }
         }
     }

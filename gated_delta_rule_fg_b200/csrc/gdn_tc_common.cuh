@@ -22,8 +22,9 @@ constexpr float kMaxHalfSpan = 6.0f;
 // vectors hit eight different bank groups.
 constexpr uint32_t kOffN = 0;            // N = -K'^T W, fp16 128x128, K-major (m=i, k=c): SBO 2048, LBO 128
 constexpr uint32_t kOffQe = 32768;       // Qe fp16 64x128 (m=r, k=c), SBO 2048, LBO 128: MN-major from intra_tc_kernel, K-major from the TMA-fed intra kernel
-constexpr uint32_t kOffB = 49152;        // b = K'^T U', fp16 [J][128][NS] (sw rows)
-constexpr uint32_t kOffPU = 81920;       // PU', fp16 [J][64][NS] (sw rows)
+constexpr uint32_t kOffB = 49152;        // b = K'^T U', fp16 [J][128][NS]: sw rows from intra_tc_kernel,
+                                         //   [J][NS / 8][128][8] from the TMA-fed intra kernel
+constexpr uint32_t kOffPU = 81920;       // PU', fp16 [J][64][NS]: sw rows / [J][NS / 8][64][8], the same way
 constexpr uint32_t kOffGC = 98304;       // e^{g_last}, fp32 [128]
 constexpr uint32_t kOffKp = 98816;       // K' fp16 (m=i, k=r), MN-major SBO 1024 LBO 128 (intra's own scratch)
 constexpr uint32_t kBlockBytes = 115200;
@@ -32,6 +33,13 @@ constexpr uint32_t kBlockBytes = 115200;
 
 __host__ __device__ __forceinline__ uint32_t sw_half(uint32_t row, uint32_t j) {
     return row * NS + 8u * (((j >> 3) ^ ((row >> 1) & 3u))) + (j & 7u);
+}
+
+// Group-major slice of `nrows` rows x 32 fp16: the 16-byte groups (8 columns) of consecutive rows
+// are consecutive, so a warp whose lanes hold consecutive rows stores and loads 512 contiguous
+// bytes per group (whole 32-byte sectors in L2, no bank conflicts in shared memory).
+__host__ __device__ __forceinline__ uint32_t grp_half(uint32_t row, uint32_t j, uint32_t nrows) {
+    return ((j >> 3) * nrows + row) * 8u + (j & 7u);
 }
 
 // swizzled fp32 64x64: element (r, i)

@@ -26,8 +26,9 @@ def off_k(mn, k, sbo, lbo):
     return (mn % 8) * 16 + (k % 8) * 2 + (mn // 8) * sbo + (k // 8) * lbo
 
 
-def sw(row, j):
-    return row * NS + 8 * ((j // 8) ^ ((row // 2) % 4)) + j % 8
+def grp(row, j, nrows):
+    # group-major slice: 16-byte groups (8 columns) of consecutive rows are consecutive
+    return ((j // 8) * nrows + row) * 8 + j % 8
 
 
 def decode(blk):
@@ -39,9 +40,9 @@ def decode(blk):
     Qe = h[(OFF_QE + off_k(r2, c3, 2048, 128)) // 2].astype(np.float64)
     jj = np.arange(128)
     bi, bj = np.meshgrid(np.arange(128), jj, indexing="ij")
-    b = h[OFF_B // 2 + (bj // NS) * 128 * NS + sw(bi, bj % NS)].astype(np.float64)
+    b = h[OFF_B // 2 + (bj // NS) * 128 * NS + grp(bi, bj % NS, 128)].astype(np.float64)
     pr, pj = np.meshgrid(np.arange(64), jj, indexing="ij")
-    PU = h[OFF_PU // 2 + (pj // NS) * 64 * NS + sw(pr, pj % NS)].astype(np.float64)
+    PU = h[OFF_PU // 2 + (pj // NS) * 64 * NS + grp(pr, pj % NS, 64)].astype(np.float64)
     gC = f[OFF_GC // 4:OFF_GC // 4 + D]
     return dict(N=N, Qe=Qe, b=b, PUp=PU, gC=gC)
 
