@@ -55,6 +55,25 @@ constexpr uint32_t kBarOff = 109056; // mbarriers (TMA, MMA), TMEM base
 constexpr uint32_t kSmem = kBarOff + 64 + 1024;   // + slack to align the base to 1024 bytes
 static_assert(2 * (kSmem + 1024) <= 233472, "two CTAs per SM");
 
+// fp32 -> tf32 (round to nearest, ties away) for the warp-level tensor-core products
+__device__ __forceinline__ uint32_t f_to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// x = hi + lo to about 2^-22 relative, both tf32
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    hi = f_to_tf32(x);
+    lo = f_to_tf32(x - __uint_as_float(hi));
+}
+// d += a b: one m16n8k8 tf32 product with fp32 accumulation (warp-wide)
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+                 "{%8, %9}, {%0, %1, %2, %3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // in-box offset of the 16-byte piece holding channels 8j .. 8j+7 (j < 8) of row r
 __device__ __forceinline__ uint32_t box16(int r, int j) {
     return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((j ^ (r & 7)) << 4));
@@ -422,12 +441,15 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     if (ok) {   // A rows -> fp32 (strictly lower), P rows -> fp16 (lower); warps w, w+4 share a lane quarter
         const int q = warp & 3, chh = warp >> 2;
         float d[32];
-        tmem_ld32(t0 + ((uint32_t)(32 * q) << 16) + 32 * chh, d);
         if (!fallback) {
             float d2[32];
-            tmem_ld32(t0 + ((uint32_t)(32 * q) << 16) + 64 + 32 * chh, d2);
+            tmem_ld32_async(t0 + ((uint32_t)(32 * q) << 16) + 32 * chh, d);
+            tmem_ld32_async(t0 + ((uint32_t)(32 * q) << 16) + 64 + 32 * chh, d2);
+            tmem_ld_wait2(d, d2);
 #pragma unroll
             for (int i = 0; i < 32; ++i) d[i] += d2[i];
+        } else {
+            tmem_ld32(t0 + ((uint32_t)(32 * q) << 16) + 32 * chh, d);
         }
         const int rho = 32 * q + lane;
         if (rho < 64) {
@@ -487,72 +509,92 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
         }
     }
     __syncthreads();
-    {   // 16x16 merges for the block pairs (16..31 | 0..15) and (48..63 | 32..47)
-        const int m = tid >> 7, qd = tid & 127;
-        const int rw = qd >> 3, j2 = (qd & 7) * 2;
-        const int bs = 32 * m;
-        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+    // Block merges T10 = -T11 (A10 T00) as warp-level tensor-core products (m16n8k8) in split
+    // tf32: every fp32 operand x = hi + lo with hi = tf32(x), lo = tf32(x - hi), and the product
+    // a b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi accumulated in fp32 (the error of the dropped
+    // a_lo b_lo term and of the splits is near fp32 rounding).  Operands are read from the fp32
+    // A / T array.  gid = lane / 4, tig = lane % 4.
+    {
+        const int gid = lane >> 2, tig = lane & 3;
+        auto Af = [&](int m0, int k0, uint32_t (&ah)[4], uint32_t (&al)[4]) {   // rows m0.., columns k0..
+            split_tf32(A32[tc::sw64(m0 + gid, k0 + tig)], ah[0], al[0]);
+            split_tf32(A32[tc::sw64(m0 + gid + 8, k0 + tig)], ah[1], al[1]);
+            split_tf32(A32[tc::sw64(m0 + gid, k0 + tig + 4)], ah[2], al[2]);
+            split_tf32(A32[tc::sw64(m0 + gid + 8, k0 + tig + 4)], ah[3], al[3]);
+        };
+        auto Bf = [&](const float* M, int ld, int k0, int n0, uint32_t (&bh)[2], uint32_t (&bl)[2], bool swz) {
+            split_tf32(swz ? M[tc::sw64(k0 + tig, n0 + gid)] : M[(k0 + tig) * ld + n0 + gid], bh[0], bl[0]);
+            split_tf32(swz ? M[tc::sw64(k0 + tig + 4, n0 + gid)] : M[(k0 + tig + 4) * ld + n0 + gid], bh[1], bl[1]);
+        };
+        // the three terms go to three accumulators (three short dependency chains), summed at the end
+        auto mma3 = [&](float (&d)[12], const uint32_t (&ah)[4], const uint32_t (&al)[4], const uint32_t (&bh)[2],
+                        const uint32_t (&bl)[2]) {
+            mma_tf32(*reinterpret_cast<float(*)[4]>(d + 8), al, bh);
+            mma_tf32(*reinterpret_cast<float(*)[4]>(d + 4), ah, bl);
+            mma_tf32(*reinterpret_cast<float(*)[4]>(d + 0), ah, bh);
+        };
+        auto sum3 = [](const float (&d)[12], int i) { return d[i] + (d[4 + i] + d[8 + i]); };
+        // 16-row merges, block pairs (16..31 | 0..15) and (48..63 | 32..47): warp w < 4 takes pair
+        // w / 2 and the 8 columns 8 (w % 2) of its 16; X = A10 T00 stays in this warp
+        if (warp < 4) {
+            const int bs = 32 * (warp >> 1), n0 = bs + 8 * (warp & 1);
+            float x[12] = {};
 #pragma unroll
-        for (int i4 = 0; i4 < 16; i4 += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(A32 + tc::sw64(bs + 16 + rw, bs + i4));
-            const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 tv = *reinterpret_cast<const float2*>(A32 + tc::sw64(bs + i4 + e, bs + j2));
-                if (e & 1) { x2 = fmaf(av[e], tv.x, x2); x3 = fmaf(av[e], tv.y, x3); }
-                else       { x0 = fmaf(av[e], tv.x, x0); x1 = fmaf(av[e], tv.y, x1); }
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                uint32_t ah[4], al[4], bh[2], bl[2];
+                Af(bs + 16, bs + k0, ah, al);
+                Bf(A32, 0, bs + k0, n0, bh, bl, true);
+                mma3(x, ah, al, bh, bl);
             }
+            float* xs = scr + warp * 128;                       // X columns n0 .. n0+7: [16][8]
+            xs[gid * 8 + 2 * tig] = sum3(x, 0);
+            xs[gid * 8 + 2 * tig + 1] = sum3(x, 1);
+            xs[(gid + 8) * 8 + 2 * tig] = sum3(x, 2);
+            xs[(gid + 8) * 8 + 2 * tig + 1] = sum3(x, 3);
+            __syncwarp();
+            float y[12] = {};
+#pragma unroll
+            for (int k0 = 0; k0 < 16; k0 += 8) {
+                uint32_t ah[4], al[4], bh[2], bl[2];
+                Af(bs + 16, bs + 16 + k0, ah, al);
+                Bf(xs, 8, k0, 0, bh, bl, false);
+                mma3(y, ah, al, bh, bl);
+            }
+            A32[tc::sw64(bs + 16 + gid, n0 + 2 * tig)] = -sum3(y, 0);
+            A32[tc::sw64(bs + 16 + gid, n0 + 2 * tig + 1)] = -sum3(y, 1);
+            A32[tc::sw64(bs + 24 + gid, n0 + 2 * tig)] = -sum3(y, 2);
+            A32[tc::sw64(bs + 24 + gid, n0 + 2 * tig + 1)] = -sum3(y, 3);
         }
-        *reinterpret_cast<float2*>(scr + m * 256 + rw * 16 + j2) = make_float2(x0 + x2, x1 + x3);
         __syncthreads();
-        float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+        // 32-row merge: T_BL = -T_BR (A_BL T_TL); warp w takes rows 32 + 16 (w / 4) and columns
+        // 8 (w % 4) of the 32 x 32 products
+        const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+        float x[12] = {};
 #pragma unroll
-        for (int m4 = 0; m4 < 16; m4 += 4) {
-            const float4 tt = *reinterpret_cast<const float4*>(A32 + tc::sw64(bs + 16 + rw, bs + 16 + m4));
-            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 xv = *reinterpret_cast<const float2*>(scr + m * 256 + (m4 + e) * 16 + j2);
-                if (e & 1) { y2 = fmaf(tv[e], xv.x, y2); y3 = fmaf(tv[e], xv.y, y3); }
-                else       { y0 = fmaf(tv[e], xv.x, y0); y1 = fmaf(tv[e], xv.y, y1); }
-            }
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            Af(32 + m0, k0, ah, al);
+            Bf(A32, 0, k0, n0, bh, bl, true);
+            mma3(x, ah, al, bh, bl);
         }
-        *reinterpret_cast<float2*>(A32 + tc::sw64(bs + 16 + rw, bs + j2)) = make_float2(-(y0 + y2), -(y1 + y3));
-    }
-    __syncthreads();
-    {   // 32x32 merge: T_BL = -T_BR (A_BL T_TL)
-        const int rw = tid >> 3, j4 = (tid & 7) * 4;
-        float4 xa = make_float4(0.f, 0.f, 0.f, 0.f), xb = xa;
-#pragma unroll
-        for (int i4 = 0; i4 < 32; i4 += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(A32 + tc::sw64(32 + rw, i4));
-            const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 tv = *reinterpret_cast<const float4*>(A32 + tc::sw64(i4 + e, j4));
-                float4& x = (e & 1) ? xb : xa;
-                x.x = fmaf(av[e], tv.x, x.x); x.y = fmaf(av[e], tv.y, x.y);
-                x.z = fmaf(av[e], tv.z, x.z); x.w = fmaf(av[e], tv.w, x.w);
-            }
-        }
-        *reinterpret_cast<float4*>(scr + 512 + rw * 32 + j4) =
-            make_float4(xa.x + xb.x, xa.y + xb.y, xa.z + xb.z, xa.w + xb.w);
+        float* xs = scr + 512;                                 // X: [32][32]
+        xs[(m0 + gid) * 32 + n0 + 2 * tig] = sum3(x, 0);
+        xs[(m0 + gid) * 32 + n0 + 2 * tig + 1] = sum3(x, 1);
+        xs[(m0 + gid + 8) * 32 + n0 + 2 * tig] = sum3(x, 2);
+        xs[(m0 + gid + 8) * 32 + n0 + 2 * tig + 1] = sum3(x, 3);
         __syncthreads();
-        float4 ya = make_float4(0.f, 0.f, 0.f, 0.f), yb = ya;
+        float y[12] = {};
 #pragma unroll
-        for (int m4 = 0; m4 < 32; m4 += 4) {
-            const float4 tt = *reinterpret_cast<const float4*>(A32 + tc::sw64(32 + rw, 32 + m4));
-            const float tv[4] = {tt.x, tt.y, tt.z, tt.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 xv = *reinterpret_cast<const float4*>(scr + 512 + (m4 + e) * 32 + j4);
-                float4& y = (e & 1) ? yb : ya;
-                y.x = fmaf(tv[e], xv.x, y.x); y.y = fmaf(tv[e], xv.y, y.y);
-                y.z = fmaf(tv[e], xv.z, y.z); y.w = fmaf(tv[e], xv.w, y.w);
-            }
+        for (int k0 = 0; k0 < 32; k0 += 8) {
+            uint32_t ah[4], al[4], bh[2], bl[2];
+            Af(32 + m0, 32 + k0, ah, al);
+            Bf(xs, 32, k0, n0, bh, bl, false);
+            mma3(y, ah, al, bh, bl);
         }
-        *reinterpret_cast<float4*>(A32 + tc::sw64(32 + rw, j4)) =
-            make_float4(-(ya.x + yb.x), -(ya.y + yb.y), -(ya.z + yb.z), -(ya.w + yb.w));
+        A32[tc::sw64(32 + m0 + gid, n0 + 2 * tig)] = -sum3(y, 0);
+        A32[tc::sw64(32 + m0 + gid, n0 + 2 * tig + 1)] = -sum3(y, 1);
+        A32[tc::sw64(40 + m0 + gid, n0 + 2 * tig)] = -sum3(y, 2);
+        A32[tc::sw64(40 + m0 + gid, n0 + 2 * tig + 1)] = -sum3(y, 3);
     }
     __syncthreads();
     for (int idx = tid; idx < 512; idx += NT) {   // T -> fp16 (rows contiguous in 16-byte pieces)
@@ -596,20 +638,20 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     if (ok) {
         const int q = warp & 3, chh = warp >> 2;
         const uint32_t lb = (uint32_t)(32 * q) << 16;
+        float d[32], dz[32];
+        tmem_ld32_async(t0 + lb + 64 + 32 * chh, d);
+        tmem_ld32_async(t0 + lb + 128 + 32 * chh, dz);
+        tmem_ld_wait2(d, dz);
         {   // Y (M = 128): row = channel, 32 columns per warp -> A operand (K-major) over A32
-            float d[32];
-            tmem_ld32(t0 + lb + 64 + 32 * chh, d);
             const int cc = 32 * q + lane;
 #pragma unroll
             for (int j = 0; j < 4; ++j) tc::st16(sm + kA32, off_kmajor(cc, 32 * chh + 8 * j, 1024, 128), tc::f_to_h8(d + 8 * j));
         }
         {   // Z (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> B operand (K-major, n = r) over T16
-            float d[32];
-            tmem_ld32(t0 + lb + 128 + 32 * chh, d);
             if (lane < 16) {
                 const int r = 16 * q + lane;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) tc::st16(sm + kT16, off_kmajor(r, 32 * chh + 8 * j, 1024, 128), tc::f_to_h8(d + 8 * j));
+                for (int j = 0; j < 4; ++j) tc::st16(sm + kT16, off_kmajor(r, 32 * chh + 8 * j, 1024, 128), tc::f_to_h8(dz + 8 * j));
             }
         }
     }
@@ -647,10 +689,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
         {   // N = -diag(row) N~ diag(col) -> block (K-major (m = i, k = c): SBO 2048, LBO 128)
             const int cc = 32 * q + lane;
             const float rs = -trow[cc];
-#pragma unroll 1
-            for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
-                float x[32];
-                tmem_ld32(t0 + lb + c0, x);
+            auto emit = [&](float (&x)[32], int c0) {
 #pragma unroll
                 for (int e4 = 0; e4 < 32; e4 += 4) {
                     const float4 cs = *reinterpret_cast<const float4*>(tcol + c0 + e4);
@@ -659,15 +698,18 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 #pragma unroll
                 for (int g8 = 0; g8 < 32; g8 += 8)
                     *reinterpret_cast<uint4*>(blk + tc::kOffN + off_kmajor(cc, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
-            }
+            };
+            float xa[32], xb[32];
+            tmem_ld32_async(t0 + lb + 64 * chh, xa);
+            tmem_ld32_async(t0 + lb + 64 * chh + 32, xb);
+            tmem_ld_wait2(xa, xb);
+            emit(xa, 64 * chh);
+            emit(xb, 64 * chh + 32);
         }
         // Qe = (QG - Z KG) diag(col) (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block
         // (K-major (m = r, k = c): SBO 2048, LBO 128)
-#pragma unroll 1
-        for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
-            float x[32];
-            tmem_ld32(t0 + lb + 128 + c0, x);
-            if (lane < 16) {
+        {
+            auto emit = [&](float (&x)[32], int c0) {
                 const int r = 16 * q + lane;
 #pragma unroll
                 for (int g8 = 0; g8 < 32; g8 += 8) {
@@ -684,6 +726,14 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
 #pragma unroll
                 for (int g8 = 0; g8 < 32; g8 += 8)
                     *reinterpret_cast<uint4*>(blk + tc::kOffQe + off_kmajor(r, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
+            };
+            float xa[32], xb[32];
+            tmem_ld32_async(t0 + lb + 128 + 64 * chh, xa);
+            tmem_ld32_async(t0 + lb + 128 + 64 * chh + 32, xb);
+            tmem_ld_wait2(xa, xb);
+            if (lane < 16) {
+                emit(xa, 64 * chh);
+                emit(xb, 64 * chh + 32);
             }
         }
     }
@@ -718,10 +768,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
         const int cc = 32 * q + lane;
         const float rs = trow[cc];
         const uint32_t lb = (uint32_t)(32 * q) << 16;
-#pragma unroll
-        for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
-            float x[32];
-            tmem_ld32(t0 + lb + c0, x);
+        auto emit = [&](float (&x)[32], int c0) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 x[e] *= rs;
@@ -730,23 +777,32 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             __half* bb = reinterpret_cast<__half*>(blk + tc::kOffB) + (size_t)(c0 / NS) * D * NS;
 #pragma unroll
             for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(bb + tc::grp_half(cc, g8, D)) = tc::f_to_h8(x + g8);
-        }
+        };
+        float xa[32], xb[32];
+        tmem_ld32_async(t0 + lb + 64 * chh, xa);
+        tmem_ld32_async(t0 + lb + 64 * chh + 32, xb);
+        tmem_ld_wait2(xa, xb);
+        emit(xa, 64 * chh);
+        emit(xb, 64 * chh + 32);
     }
     if (ok) {   // PU' (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (fp16 group-major slices)
         const int q = warp & 3, chh = warp >> 2;
         const uint32_t lb = (uint32_t)(32 * q) << 16;
-#pragma unroll 1
-        for (int c0 = 64 * chh; c0 < 64 * chh + 64; c0 += 32) {
-            float x[32];
-            tmem_ld32(t0 + lb + 128 + c0, x);
-            if (lane < 16) {
-                const int r = 16 * q + lane;
-                __half* pu = reinterpret_cast<__half*>(blk + tc::kOffPU) + (size_t)(c0 / NS) * C * NS;
+        auto emit = [&](float (&x)[32], int c0) {
+            const int r = 16 * q + lane;
+            __half* pu = reinterpret_cast<__half*>(blk + tc::kOffPU) + (size_t)(c0 / NS) * C * NS;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) vmax = fmax_nan(vmax, fabsf(x[e]));
+            for (int e = 0; e < 32; ++e) vmax = fmax_nan(vmax, fabsf(x[e]));
 #pragma unroll
-                for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::grp_half(r, g8, C)) = tc::f_to_h8(x + g8);
-            }
+            for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::grp_half(r, g8, C)) = tc::f_to_h8(x + g8);
+        };
+        float xa[32], xb[32];
+        tmem_ld32_async(t0 + lb + 128 + 64 * chh, xa);
+        tmem_ld32_async(t0 + lb + 128 + 64 * chh + 32, xb);
+        tmem_ld_wait2(xa, xb);
+        if (lane < 16) {
+            emit(xa, 64 * chh);
+            emit(xb, 64 * chh + 32);
         }
     }
     if (tid < D) reinterpret_cast<float*>(blk + tc::kOffGC)[tid] = tgam[tid];
