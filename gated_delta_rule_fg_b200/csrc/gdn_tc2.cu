@@ -232,12 +232,14 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     // exclusive prefix of the row-group totals per channel, and gamma
     bool wide = false;
     if (tid < D) {
+        float v[16];                      // all sixteen loads first, then the dependent products
+#pragma unroll
+        for (int g = 0; g < 16; ++g) v[g] = scr[g * D + tid];
         float acc = 1.f;
 #pragma unroll
         for (int g = 0; g < 16; ++g) {
-            const float v = scr[g * D + tid];
             scr[g * D + tid] = acc;
-            acc *= v;
+            acc *= v[g];
         }
         tgam[tid] = acc;
         wide = !(acc >= kMinGamma);
@@ -257,17 +259,14 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     __half* fb_k = reinterpret_cast<__half*>(blk + tc::kOffPU);               // k~ fp16 [C][D]
     __half* fb_q = reinterpret_cast<__half*>(blk + tc::kOffN);                // q^ fp16 [C][D]
     if (!fallback) {
-        float pre[8], rf[8], iv[8];
+        float pre[8];       // the row group's prefix, over ref: P = pre * lp * ref
         {
             const float4 a0 = *reinterpret_cast<const float4*>(scr + rg * D + ch0);
             const float4 a1 = *reinterpret_cast<const float4*>(scr + rg * D + ch0 + 4);
             pre[0] = a0.x; pre[1] = a0.y; pre[2] = a0.z; pre[3] = a0.w;
             pre[4] = a1.x; pre[5] = a1.y; pre[6] = a1.z; pre[7] = a1.w;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                rf[e] = tref[ch0 + e];
-                iv[e] = tinv[ch0 + e];
-            }
+            for (int e = 0; e < 8; ++e) pre[e] *= tinv[ch0 + e];
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -293,13 +292,13 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             float KG[8], QG[8], KI[8], VT[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float P = pre[e] * lp[i][e];
-                const float rp = __fdividef(1.f, P);     // P >= gamma >= e^{-12}: no overflow
+                const float Pv = pre[e] * lp[i][e];      // P / ref, in [e^{-6}, e^{6}]
+                const float rpv = __fdividef(1.f, Pv);   // ref / P
                 const float sb = tc::sqrt_op(be[i][e]);
                 const float kt = fk[e] * ik[i] * sb;
-                KG[e] = kt * (P * iv[e]);
-                KI[e] = kt * (rf[e] * rp);
-                QG[e] = fq[e] * iq[i] * (P * iv[e]);
+                KG[e] = kt * Pv;
+                KI[e] = kt * rpv;
+                QG[e] = fq[e] * iq[i] * Pv;
                 VT[e] = fv[e] * (kPlus ? sv[e] : sb);
                 vmax = fmax_nan(vmax, fabsf(VT[e]));
             }
