@@ -367,6 +367,7 @@ gdn_status_t gdn_workspace_status(void* workspace, cudaStream_t stream) {
         case 0: return GDN_OK;
         case kDevTimeout: return GDN_ERR_TIMEOUT;
         case kDevRange: return GDN_ERR_RANGE;
+        case kDevBounds: return GDN_ERR_BOUNDS;
         default: return GDN_ERR_CUDA;
     }
 }
@@ -380,6 +381,7 @@ const char* gdn_status_string(gdn_status_t s) {
         case GDN_ERR_TIMEOUT: return "device wait timed out";
         case GDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
         case GDN_ERR_RANGE: return "value outside the fp16 operand range";
+        case GDN_ERR_BOUNDS: return "index outside its buffer (bounds-checking build)";
     }
     return "unknown status";
 }

@@ -82,6 +82,7 @@ template <typename Tin, int NR, int NI>
 __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
     const int j0 = blockIdx.x * kNS;
     const int bh = blockIdx.y;
+    if (!GDN_IN_BOUNDS(j0 + kNS <= p.dv && bh < p.B * p.H, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int tid = threadIdx.x;
@@ -210,6 +211,7 @@ template <typename Tin, int RPT>
 __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int s0 = c * C;

@@ -33,7 +33,20 @@
 namespace gdn {
 
 // Device-side error codes recorded in the workspace header (match gdn_status_t).
-enum : int { kDevOk = 0, kDevTimeout = 4, kDevRange = 6 };
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevRange = 6, kDevBounds = 7 };
+
+// Bounds checks of the bounds-checking build (-DGDN_DEBUG_BOUNDS): GDN_IN_BOUNDS(cond, status)
+// is false, and GDN_ERR_BOUNDS is recorded in the workspace status word, when `cond` does not
+// hold; the caller then skips the access.  In the normal build it is the constant true.
+#ifdef GDN_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool cond, int* status) {
+    if (!cond) atomicCAS(status, (int)kDevOk, (int)kDevBounds);
+    return cond;
+}
+#define GDN_IN_BOUNDS(cond, status) (::gdn::bounds_ok((cond), (status)))
+#else
+#define GDN_IN_BOUNDS(cond, status) true
+#endif
 
 struct Problem {
     const void* q;

@@ -31,7 +31,16 @@ using tc::NS;
 template <int W>
 struct Cfg {
     static constexpr int NSW = NS * W;                       // columns of this CTA
-    static constexpr int kThreads = 32 * (4 * W + 12);
+    // Warp roles.  A warp reads and writes the tensor-memory lanes of quarter warp % 4, which
+    // fixes where the Qe feeders and output writers sit.  One slice: Qe rows 0 .. 63 go to lanes
+    // 64 .. 127 only (quarters 2, 3); two slices: to both lane halves (quarters 0 .. 3), and the
+    // outputs of slice 0 are read from lanes 64 .. 127, those of slice 1 from lanes 0 .. 63.
+    static constexpr int kNFeed0 = 4 * W;                    // 4 N feeders
+    static constexpr int kQe0 = W == 1 ? 10 : 12, kNQe = W == 1 ? 2 : 4;
+    static constexpr int kOut0 = W == 1 ? 14 : 16, kNOut = W == 1 ? 2 : 4;
+    static constexpr int kProducer = W == 1 ? 8 : 20, kMmaS = W == 1 ? 9 : 21, kMmaO = W == 1 ? 12 : 22;
+    static constexpr int kWarps = W == 1 ? 16 : 23;
+    static constexpr int kThreads = 32 * kWarps;
     // Three rings, each released by the role that reads it last: {N, Qe} by the feeders once
     // copied into tensor memory, {b slices, gC} by the state warps, {PU' slices} by the output
     // warps (which run two chunks behind the chain, so their data must not hold back the state
@@ -64,6 +73,8 @@ static_assert(Cfg<1>::kRingBG % 128 == 0 && Cfg<1>::kRingPU % 128 == 0 && Cfg<1>
 static_assert(Cfg<2>::kRingBG % 128 == 0 && Cfg<2>::kRingPU % 128 == 0 && Cfg<2>::kSop % 128 == 0, "alignment");
 static_assert(Cfg<1>::kSmem <= 227 * 1024 && Cfg<2>::kSmem <= 227 * 1024, "shared memory");
 static_assert(Cfg<1>::kTN + 128 <= 512 && Cfg<2>::kTN + 128 <= 512, "tensor memory");
+static_assert(Cfg<1>::kQe0 % 4 == 2 && Cfg<1>::kOut0 % 4 == 2 && Cfg<2>::kQe0 % 4 == 0 && Cfg<2>::kOut0 % 4 == 0,
+              "Qe feeders and output writers on the lane quarters they use");
 
 // Copies rows of a K-major (SBO 2048, LBO 128) fp16 tile from shared memory into tensor memory
 // as an A operand: this thread's row `row`, 128 fp16 = 64 columns, lane = row.
@@ -108,6 +119,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (!GDN_IN_BOUNDS(cb >= 0 && ce <= p.NC && bh < p.B * p.H && slice0 + W <= tc::J, p.status)) return;
     uint64_t* fullNQ = reinterpret_cast<uint64_t*>(sm + kBar);
     uint64_t* emptyNQ = fullNQ + kNQ;
     uint64_t* fullBG = emptyNQ + kNQ;
@@ -134,9 +146,9 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < kNQ; ++i) { mbar_init(&fullNQ[i], 1); mbar_init(&emptyNQ[i], 4 + 2); }
+        for (int i = 0; i < kNQ; ++i) { mbar_init(&fullNQ[i], 1); mbar_init(&emptyNQ[i], 4 + K::kNQe); }
         for (int i = 0; i < kBG; ++i) { mbar_init(&fullBG[i], 1); mbar_init(&emptyBG[i], 4 * W); }
-        for (int i = 0; i < kPU; ++i) { mbar_init(&fullPU[i], 1); mbar_init(&emptyPU[i], 2); }
+        for (int i = 0; i < kPU; ++i) { mbar_init(&fullPU[i], 1); mbar_init(&emptyPU[i], K::kNOut); }
         mbar_init(bar_s, 1);
         mbar_init(s_ready, 4 * W);
         for (int i = 0; i < 2; ++i) {
@@ -144,10 +156,10 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             mbar_init(&n_free[i], 1);
         }
         for (int i = 0; i < kNO; ++i) {
-            mbar_init(&q_ready[i], 2);
+            mbar_init(&q_ready[i], K::kNQe);
             mbar_init(&q_free[i], 1);
             mbar_init(&bar_o[i], 1);
-            mbar_init(&o_free[i], 2);
+            mbar_init(&o_free[i], K::kNOut);
         }
         for (int i = 0; i < kSl; ++i) {
             mbar_init(&s_slot[i], 4 * W);
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
     const uint64_t lim = p.test_wait_ns ? p.test_wait_ns : kWaitLimitNs;
     bool ok = true;
 
-    if (warp == 4 * W + 4) {
+    if (warp == K::kProducer) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             // The rings are only a few chunks deep, less than a DRAM round trip at the chain's
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             for (int i = 0; i < kPU; ++i)
                 if (ld_pu[i] >= 0) mbar_wait(&fullPU[i], (ld_pu[i] / kPU) & 1, lim);
         }
-    } else if (warp == 4 * W + 5) {
+    } else if (warp == K::kMmaS) {
         // ------------------------------------------------------------ chain MMA issuer (one thread)
         // A thread that issues tcgen05.mma is held for about the time the tensor pipe takes to
         // accept each instruction, while two issuing threads proceed side by side; so the chain
@@ -239,7 +251,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             mma_commit(bar_d);
             if (!mbar_wait(bar_d, 0, lim)) tc::record_timeout(p.status);
         }
-    } else if (warp == 4 * W + 8) {
+    } else if (warp == K::kMmaO) {
         // ------------------------------------------------------------ output MMA issuer (one thread)
         // MMA_O(c) reads S_c from Sop slot c % kSl once the state warps have written it; its
         // completion (o_done) lets them write S_{c+kSl} there.
@@ -287,18 +299,9 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             const uint8_t* bp = sm + kRingBG + sb * kBGBytes;
             if (!__all_sync(0xffffffffu, mbar_wait(&fullBG[sb], (ch / kBG) & 1, lim))) { ok = false; break; }
             const __half* bsm = reinterpret_cast<const __half*>(bp) + sl * (D * NS);
-            float bv[NS];
+            uint4 bq[NS / 8];                                  // b, kept as fp16 pairs until used
 #pragma unroll
-            for (int g8 = 0; g8 < NS; g8 += 8) {
-                const uint4 v = *reinterpret_cast<const uint4*>(bsm + tc::grp_half(row, g8, D));
-                const __half2* hh = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __half22float2(hh[e]);
-                    bv[g8 + 2 * e] = f.x;
-                    bv[g8 + 2 * e + 1] = f.y;
-                }
-            }
+            for (int g8 = 0; g8 < NS; g8 += 8) bq[g8 / 8] = *reinterpret_cast<const uint4*>(bsm + tc::grp_half(row, g8, D));
             const float gc = reinterpret_cast<const float*>(bp + 8192 * W)[row];
             // Sop slot (ch + 1) % kSl last held S_{ch+1-kSl}: its output product must be done before
             // S_{ch+1} goes there (its chain product is: MMA_S(ch) completes after it).  Checked
@@ -313,7 +316,15 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             float d[NS];
             tmem_ld32(t0 + kTS + lanebase + NS * sl, d);
 #pragma unroll
-            for (int j = 0; j < NS; ++j) S[j] = fmaf(gc, S[j], d[j] + bv[j]);
+            for (int g8 = 0; g8 < NS; g8 += 8) {
+                const __half2* hh = reinterpret_cast<const __half2*>(&bq[g8 / 8]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(hh[e]);
+                    S[g8 + 2 * e] = fmaf(gc, S[g8 + 2 * e], d[g8 + 2 * e] + f.x);
+                    S[g8 + 2 * e + 1] = fmaf(gc, S[g8 + 2 * e + 1], d[g8 + 2 * e + 1] + f.y);
+                }
+            }
             uint8_t* snext = sm + kSop + ((ch + 1) % kSl) * kSopBytes;
 #pragma unroll
             for (int j = 0; j < NS; j += 8) tc::st16(snext, off_mnmajor(NS * sl + j, row, 2048, 128), tc::f_to_h8(S + j));
@@ -336,9 +347,9 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
 #pragma unroll
             for (int j = 0; j < NS; j += 4) dst[j / 4] = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
         }
-    } else if (warp < 4 * W + 4) {
-        // ------------------------------------------------------------ N feeders (warps 4W .. 4W+3)
-        const int q = warp - 4 * W;                            // TMEM lane quarter
+    } else if (warp >= K::kNFeed0 && warp < K::kNFeed0 + 4) {
+        // ------------------------------------------------------------ N feeders
+        const int q = warp - K::kNFeed0;                       // TMEM lane quarter
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
         const int row = 32 * q + lane;
         // N_c into buffer c & 1 once MMA_S(c - 2) has read it
@@ -357,11 +368,11 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             }
         }
         if (!ok && lane == 0) tc::record_timeout(p.status);
-    } else if (warp < 4 * W + 8) {
-        // ------------------------------------------------------------ Qe feeders (warps 4W+6, 4W+7)
-        const int q = warp & 3;                                // TMEM lane quarter: 2 or 3
+    } else if (warp >= K::kQe0 && warp < K::kQe0 + K::kNQe) {
+        // ------------------------------------------------------------ Qe feeders
+        const int q = warp & 3;                                // TMEM lane quarter
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-        const int row = 32 * (q - 2) + lane;                   // Qe row of the chunk
+        const int row = 32 * (q & 1) + lane;                   // Qe row of the chunk
         // Qe_it into buffer it % kNO (lanes 64 .. 127) once MMA_O(it - kNO) has read it
         for (int it = 0; it < nloc && ok; ++it) {
             const int s2 = it % kNQ;
@@ -379,11 +390,12 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             }
         }
         if (!ok && lane == 0) tc::record_timeout(p.status);
-    } else if (warp >= 4 * W + 10) {
-        // ------------------------------------------------------------ outputs (warps 4W+10, 4W+11)
-        const int q = warp & 3;                                // TMEM lane quarter: 2 or 3
+    } else if (warp >= K::kOut0 && warp < K::kOut0 + K::kNOut) {
+        // ------------------------------------------------------------ output writers
+        const int q = warp & 3;                                // TMEM lane quarter
         const uint32_t lanebase = (uint32_t)(32 * q) << 16;
-        const int row = 32 * (q - 2) + lane;                   // output row of the chunk (D_O lane 64 + row)
+        const int row = 32 * (q & 1) + lane;                   // output row of the chunk
+        const int sl = W == 1 ? 0 : 1 - (q >> 1);              // slice: lanes 64-127 slice 0, 0-63 slice 1
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
         for (int oc = 0; oc < nloc && ok; ++oc) {
             const int sp = oc % kPU;
@@ -393,16 +405,14 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
             tc_fence_after();
             const int s = (cb + oc) * C + row;
             RowRef ro{};
-            const bool write = s < p.L && (ro = row_ref(p, b, h, s)).has_q;
-#pragma unroll 1
-            for (int sl = 0; sl < W; ++sl) {
+            const bool write = s < p.L && (ro = row_ref(p, b, h, s)).has_q &&
+                               GDN_IN_BOUNDS(ro.tok < (size_t)p.B * p.T * p.H, p.status);
+            {
                 float d[NS];
                 tmem_ld32(t0 + kTO + NSW * bo + NS * sl + lanebase, d);
-                if (sl == W - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&o_free[bo]);
-                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&o_free[bo]);
                 if (write) {
                     const __half* pu = reinterpret_cast<const __half*>(sm + kRingPU + sp * kPUBytes) + sl * (C * NS);
                     uint4* dst = reinterpret_cast<uint4*>(out + ro.tok * D + (slice0 + sl) * NS);

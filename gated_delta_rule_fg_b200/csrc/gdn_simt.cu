@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 intra_simt_kernel(Problem p) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;   // the whole CTA, before any barrier
     const int b = bh / p.H, h = bh % p.H;
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int s0 = c * C;
@@ -267,6 +268,7 @@ __global__ void __launch_bounds__(kSimtThreads)
 scan_simt_kernel(Problem p) {
     const int j0 = blockIdx.x * kScanCols;
     const int bh = blockIdx.y;
+    if (!GDN_IN_BOUNDS(j0 + kScanCols <= p.dv && bh < p.B * p.H, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int tid = threadIdx.x;

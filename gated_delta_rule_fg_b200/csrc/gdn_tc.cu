@@ -29,6 +29,7 @@
 //
 // launch_tc cuts long sequences into chunk ranges: intra of range s+1 runs on
 // the caller's stream while the scan of range s runs on the side stream.
+#include <cstdlib>
 #include <mutex>
 
 #include "gdn_tc_common.cuh"
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tc_kernel(Problem p, int cb) {
     const int s0 = c * C;
     const int Cv = min(C, p.L - s0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;   // the whole CTA, before any barrier
     uint8_t* blk = static_cast<uint8_t*>(p.inter) + ((size_t)bh * p.NC + c) * kBlockBytes;
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kBar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kTmem);
@@ -780,6 +782,7 @@ __global__ void __launch_bounds__(ScanCfg<W>::kThreads, 1) scan_tc_kernel(Proble
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (!GDN_IN_BOUNDS(cb >= 0 && ce <= p.NC && bh < p.B * p.H && slice0 + W <= J, p.status)) return;
     uint64_t* fullNB = reinterpret_cast<uint64_t*>(sm + Cfg::kSBar);
     uint64_t* emptyNB = fullNB + kNB;
     uint64_t* fullQP = emptyNB + kNB;
@@ -1039,6 +1042,18 @@ cudaError_t launch_intra_tma(const Problem& p, int cb, int n, cudaStream_t strea
 cudaError_t launch_scan2(const Problem& p, int cb, int ce, const float* S_in, float* S_out, cudaStream_t stream);
 
 cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
+#ifdef GDN_DEBUG_BOUNDS
+    // Test knob of the bounds-checking build only (environment GDN_TEST_BOUNDS_NC_OFF=1): the
+    // kernels are told one chunk fewer than their grids cover, so the checks on the last chunk's
+    // CTAs fire (and skip their accesses); the block stride shrinks with it, so every address
+    // formed stays inside the workspace.
+    Problem pk_ = p;
+    if (const char* e = std::getenv("GDN_TEST_BOUNDS_NC_OFF"))
+        if (e[0] == '1' && pk_.NC > 1) pk_.NC -= 1;
+    const Problem& pk = pk_;
+#else
+    const Problem& pk = p;
+#endif
     auto intra = p.gdn2_eta ? tc::intra_tc_kernel<false, true>
                : (p.beta_v ? tc::intra_tc_kernel<true> : tc::intra_tc_kernel<false>);
     const bool tma = tc2_usable(p);
@@ -1049,8 +1064,8 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     }
     // intra role over chunks [cb, cb + n) of every head
     auto launch_intra = [&](int cb, int n, cudaStream_t st) -> cudaError_t {
-        if (tma) return launch_intra_tma(p, cb, n, st);
-        intra<<<dim3(n, p.B * p.H), tc::NT, tc::kIntraSmem, st>>>(p, cb);
+        if (tma) return launch_intra_tma(pk, cb, n, st);
+        intra<<<dim3(n, p.B * p.H), tc::NT, tc::kIntraSmem, st>>>(pk, cb);
         return cudaGetLastError();
     };
     // scan width: two slices per CTA when one slice per CTA would take more than one wave
@@ -1069,8 +1084,8 @@ cudaError_t launch_tc(const Problem& p, cudaStream_t stream) {
     const int P = tc_segments(p);
     // scan role over chunks [cb, ce)
     auto launch_scan = [&](int cb, int ce, const float* S_in, float* S_out, cudaStream_t st) -> cudaError_t {
-        if (tma) return launch_scan2(p, cb, ce, S_in, S_out, st);
-        scan<<<g2, scan_threads, scan_smem, st>>>(p, cb, ce, S_in, S_out);
+        if (tma) return launch_scan2(pk, cb, ce, S_in, S_out, st);
+        scan<<<g2, scan_threads, scan_smem, st>>>(pk, cb, ce, S_in, S_out);
         return cudaGetLastError();
     };
     auto one_stream = [&]() {               // both roles over all chunks, on the caller's stream

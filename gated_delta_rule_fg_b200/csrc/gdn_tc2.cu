@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
     const int s0 = c * C;
     const int Cv = min(C, p.L - s0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;   // the whole CTA, before any barrier
     uint8_t* blk = static_cast<uint8_t*>(p.inter) + ((size_t)bh * p.NC + c) * tc::kBlockBytes;
     uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + kBarOff);
     uint64_t* bar_mma = bar_tma + 1;
@@ -166,21 +167,22 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, con
             continue;
         }
         tok = ((size_t)b * p.T + s0 + r) * p.H + h;
-        if (valid && !a_scalar) {
+        const bool vr = valid && GDN_IN_BOUNDS(tok < (size_t)p.B * p.T * p.H, p.status);
+        if (vr && !a_scalar) {
             const float4 x0 = tc::ldg16f(p.alpha + tok * D + ch0), x1 = tc::ldg16f(p.alpha + tok * D + ch0 + 4);
             lp[i][0] = x0.x; lp[i][1] = x0.y; lp[i][2] = x0.z; lp[i][3] = x0.w;
             lp[i][4] = x1.x; lp[i][5] = x1.y; lp[i][6] = x1.z; lp[i][7] = x1.w;
         } else {
-            const float a = valid ? __ldg(p.alpha + tok) : 1.f;
+            const float a = vr ? __ldg(p.alpha + tok) : 1.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) lp[i][e] = a;
         }
-        if (valid && !b_scalar) {
+        if (vr && !b_scalar) {
             const float4 x0 = tc::ldg16f(p.beta + tok * D + ch0), x1 = tc::ldg16f(p.beta + tok * D + ch0 + 4);
             be[i][0] = x0.x; be[i][1] = x0.y; be[i][2] = x0.z; be[i][3] = x0.w;
             be[i][4] = x1.x; be[i][5] = x1.y; be[i][6] = x1.z; be[i][7] = x1.w;
         } else {
-            const float bb = valid ? __ldg(p.beta + tok) : 0.f;
+            const float bb = vr ? __ldg(p.beta + tok) : 0.f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) be[i][e] = bb;
         }

@@ -14,9 +14,14 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
+# GDN_DEBUG_BOUNDS=1 in the environment selects the bounds-checking build of the same library
+# (built by `python -m gated_delta_rule_fg_b200.build --debug-bounds`).
+BOUNDS_LIB_PATH = os.path.join(_HERE, "libgdn_b200_bounds.so")
+if os.environ.get("GDN_DEBUG_BOUNDS", "") not in ("", "0"):
+    LIB_PATH = BOUNDS_LIB_PATH
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, 1, 2, 3
-GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE, GDN_ERR_RANGE = 4, 5, 6
+GDN_ERR_TIMEOUT, GDN_ERR_WORKSPACE, GDN_ERR_RANGE, GDN_ERR_BOUNDS = 4, 5, 6, 7
 GDN_F32, GDN_BF16 = 0, 1
 GDN_ALPHA_SCALAR, GDN_BETA_SCALAR, GDN_SINGLE_STREAM = 1, 2, 4
 

@@ -83,7 +83,9 @@ typedef enum {
     GDN_ERR_CUDA = 3,          /* a CUDA launch or copy failed (cudaGetLastError is left set) */
     GDN_ERR_TIMEOUT = 4,       /* device side: a bounded wait ran out; outputs are not valid */
     GDN_ERR_WORKSPACE = 5,     /* workspace NULL, misaligned or smaller than required */
-    GDN_ERR_RANGE = 6          /* device side: a value left the fp16 operand range of the tensor-core path */
+    GDN_ERR_RANGE = 6,         /* device side: a value left the fp16 operand range of the tensor-core path */
+    GDN_ERR_BOUNDS = 7         /* device side, bounds-checking build only: an index left its buffer
+                                  (the access was skipped; outputs are not valid) */
 } gdn_status_t;
 
 typedef enum {
@@ -304,8 +306,15 @@ gdn_status_t gdn_recurrent_step(const void* q, const void* k, const void* v,
                                 cudaStream_t stream);
 
 /* Waits for `stream`, then returns (and clears) the first device-side error
- * recorded in `workspace` by earlier calls: GDN_OK, GDN_ERR_TIMEOUT or
- * GDN_ERR_RANGE; GDN_ERR_CUDA if the wait itself failed.
+ * recorded in `workspace` by earlier calls: GDN_OK, GDN_ERR_TIMEOUT,
+ * GDN_ERR_RANGE or (bounds-checking build) GDN_ERR_BOUNDS; GDN_ERR_CUDA if the
+ * wait itself failed.
+ *
+ * Bounds-checking build: the library compiled with -DGDN_DEBUG_BOUNDS
+ * (libgdn_b200_bounds.so; `python -m gated_delta_rule_fg_b200.build
+ * --debug-bounds`) checks the global-memory indices its kernels form against
+ * the extents of the buffers they address; an index outside records
+ * GDN_ERR_BOUNDS and the access is skipped instead of faulting.  Same ABI.
  *
  * Every device-side wait of the library is bounded (2 s); a wait that runs out
  * records GDN_ERR_TIMEOUT and the kernel unwinds (its copies land, its tensor

@@ -39,9 +39,24 @@ def test_exports_every_declared_symbol(L):
 
 def test_version_and_status_strings(L):
     assert L.gdn_version() >= 100
-    for code in range(7):
+    for code in range(8):
         assert len(ops.status_string(code)) > 0
+    assert ops.status_string(ops.GDN_ERR_BOUNDS) != "unknown status"
     assert ops.status_string(99) == "unknown status"
+
+
+def test_bounds_checking_build_exports_the_same_abi():
+    """The bounds-checking build (-DGDN_DEBUG_BOUNDS) is the same ABI in another file."""
+    from gated_delta_rule_fg_b200 import build
+    path = build.build(debug_bounds=True)
+    assert path == ops.BOUNDS_LIB_PATH and os.path.exists(path)
+    B = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(B, n), f"{n} declared in gdn.h but not exported by the bounds-checking build"
+    B.gdn_chunk_fwd_workspace_size.restype = ctypes.c_size_t
+    B.gdn_chunk_fwd_workspace_size.argtypes = ops.SIGNATURES["gdn_chunk_fwd_workspace_size"][1]
+    assert B.gdn_chunk_fwd_workspace_size(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0) == \
+        ops.chunk_fwd_workspace_size(1, 16, 32768, 128, 128, 64, ops.GDN_BF16, 0)
 
 
 def test_workspace_sizes(L):
