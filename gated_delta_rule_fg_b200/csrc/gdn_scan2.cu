@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(Cfg<W>::kThreads, 1) scan2_kernel(Problem p, i
         if (lane == 0) {
             // The rings are only a few chunks deep, less than a DRAM round trip at the chain's
             // pace, so the blocks kPrefetch chunks ahead are first pulled into L2.
-            constexpr int kPrefetch = 8;
+            constexpr int kPrefetch = 4;
             auto prefetch = [&](int ch) {
                 const uint8_t* src = blocks + (size_t)(cb + ch) * tc::kBlockBytes;
                 bulk_prefetch_l2(src + tc::kOffN, 32768 + 16384);                       // N, Qe
