@@ -477,7 +477,9 @@ def main():
     barrier()
     clk = clocks.stop() if not args.profile else None
     total_ms = e0.elapsed_time(e1)
-    per_call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    call_ms = [a.elapsed_time(b) for a, b in ev]
+    per_call_ms = float(np.mean(call_ms))
+    per_call_ms_median = float(np.median(call_ms))
     if ws is not None:
         status = ops.workspace_status(ws)
         if status != ops.GDN_OK:
@@ -548,7 +550,7 @@ def main():
             "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": op.flops,
             "flop_frac_of_bf16_peak": op.flops / (per_call_ms / 1000.0) / (bf16_tf * 1e12),
             "flop_frac_of_bf16_sustained": op.flops / (per_call_ms / 1000.0) / (bf16_tf_sus * 1e12),
-            "launch_ms": per_call_ms}
+            "launch_ms": per_call_ms, "launch_ms_median": per_call_ms_median}
 
     line = {"metric": op.metric, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

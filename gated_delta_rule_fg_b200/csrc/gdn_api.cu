@@ -138,6 +138,16 @@ int gdn_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, gdn_d
     return launches_for(p, dtype == GDN_BF16);
 }
 
+int gdn_chunk_fwd_tensor_cores(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                               unsigned flags) {
+    Problem p;
+    if (make_problem(p, B, H, T, 1, dk, dv, chunk, dtype, flags, false) != GDN_OK) return -1;
+    // (T == 0 and empty batches enqueue no chunk work; the answer is the path the sizes select)
+    Problem q = p;
+    if (q.T == 0) q.T = 1;
+    return tc_supported(q, dtype == GDN_BF16) ? 1 : 0;
+}
+
 int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
                                   gdn_dtype_t dtype) {
     Problem p;

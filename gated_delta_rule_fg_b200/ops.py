@@ -43,6 +43,7 @@ SIGNATURES = {
     "gdn_deltaproduct_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                   _I, _P, _SZ, _P]),
     "gdn_chunk_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
+    "gdn_chunk_fwd_tensor_cores": (_I, [_I, _I, _I, _I, _I, _I, _I, ctypes.c_uint]),
     "gdn_deltaproduct_fwd_launches": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gdn_recurrent_step": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                                 ctypes.c_uint, _P]),
@@ -112,6 +113,12 @@ def _check(t, name, dtype=None):
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def chunk_fwd_tensor_cores(B, H, T, dk, dv, chunk, dtype_code, flags=0) -> int:
+    """1: gdn_chunk_fwd takes the tensor-core path for these sizes; 0: the float32 CUDA-core
+    path; -1: invalid or unsupported sizes."""
+    return int(lib().gdn_chunk_fwd_tensor_cores(B, H, T, dk, dv, chunk, dtype_code, flags))
 
 
 def chunk_fwd_workspace_size(B, H, T, dk, dv, chunk, dtype_code, flags) -> int:

@@ -209,6 +209,13 @@ int gdn_plus_chunk_fwd_launches(int B, int H, int T, int dk, int dv, int chunk, 
 int gdn_deltaproduct_fwd_launches(int B, int H, int T, int n_h, int dk, int dv, int chunk,
                                   gdn_dtype_t dtype);
 
+/* Which path a gdn_chunk_fwd call with these sizes takes: 1 the tensor-core path (tcgen05,
+ * fp16 operands, fp32 accumulation), 0 the float32 CUDA-core path (a few tens of times slower
+ * at the same size), -1 invalid or unsupported sizes.  The tensor-core path takes GDN_BF16
+ * with dk == dv == 128 and chunk 64 (or 128). */
+int gdn_chunk_fwd_tensor_cores(int B, int H, int T, int dk, int dv, int chunk, gdn_dtype_t dtype,
+                               unsigned flags);
+
 /* GDN2 transform modes (Su Jianlin's GDN2 stability note): none; clip the decay to
  * min(D, 1/rho) with rho the closed-form spectral norm of I - j' k^T ("Simple
  * Strategy"); or shrink j' toward KDA keeping j'^T k ("Modifying Itself"). */

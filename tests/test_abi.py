@@ -45,6 +45,19 @@ def test_version_and_status_strings(L):
     assert ops.status_string(99) == "unknown status"
 
 
+def test_path_query(L):
+    """gdn_chunk_fwd_tensor_cores says which path a call takes (no device access)."""
+    tc = ops.chunk_fwd_tensor_cores
+    assert tc(1, 16, 32768, 128, 128, 64, ops.GDN_BF16) == 1
+    assert tc(1, 16, 32768, 128, 128, 128, ops.GDN_BF16) == 1      # chunk 128: 64-row chunks
+    assert tc(1, 2, 0, 128, 128, 64, ops.GDN_BF16) == 1             # empty sequence: same path
+    assert tc(1, 16, 4096, 128, 128, 32, ops.GDN_BF16) == 0         # chunk 32: CUDA cores
+    assert tc(1, 16, 4096, 64, 64, 64, ops.GDN_BF16) == 0           # d 64: CUDA cores
+    assert tc(1, 16, 4096, 64, 64, 64, ops.GDN_F32) == 0            # float32: CUDA cores
+    assert tc(1, 16, 4096, 96, 96, 64, ops.GDN_BF16) == -1          # unsupported head dim
+    assert tc(1, 16, 4096, 128, 128, 48, ops.GDN_BF16) == -1        # unsupported chunk
+
+
 def test_bounds_checking_build_exports_the_same_abi():
     """The bounds-checking build (-DGDN_DEBUG_BOUNDS) is the same ABI in another file."""
     from gated_delta_rule_fg_b200 import build
