@@ -84,13 +84,16 @@ __device__ __forceinline__ uint32_t box16(int r, int j) {
 // 5-D maps (channel, step, head, token, batch) whose boxes are whole tokens, and q (one row per
 // token, on its last step) is read with vector loads.
 template <bool kPlus, bool kDP>
-__global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, const __grid_constant__ CUtensorMap tmq,
+__global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int head_fastest,
+                                                          const __grid_constant__ CUtensorMap tmq,
                                                           const __grid_constant__ CUtensorMap tmk,
                                                           const __grid_constant__ CUtensorMap tmv) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
-    const int c = cb + blockIdx.x;
-    const int bh = blockIdx.y;
+    // head_fastest: blockIdx.x is the head, so CTAs launched together read the same token rows
+    // (adjacent in memory) for different heads
+    const int c = cb + (head_fastest ? blockIdx.y : blockIdx.x);
+    const int bh = head_fastest ? blockIdx.x : blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int s0 = c * C;
     const int Cv = min(C, p.L - s0);
@@ -881,7 +884,8 @@ cudaError_t launch_intra_tma(const Problem& p, int cb, int n, cudaStream_t strea
               : (p.beta_v ? tc2::intra_tma_kernel<true, false> : tc2::intra_tma_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc2::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(n, p.B * p.H), tc2::NT, tc2::kSmem, stream>>>(p, cb, mq, mk, mv);
+    const int hf = n <= 65535 ? 1 : 0;                 // grid y is at most 65535
+    kern<<<hf ? dim3(p.B * p.H, n) : dim3(n, p.B * p.H), tc2::NT, tc2::kSmem, stream>>>(p, cb, hf, mq, mk, mv);
     return cudaGetLastError();
 }
 

@@ -163,7 +163,7 @@ def test_tensor_core_shapes_modes(mode, T):
     check(cfg, run_gdn(cfg, x), oracle_gdn(cfg, x))
 
 
-@pytest.mark.parametrize("nh,T", [(2, 100), (3, 70), (1, 130)])
+@pytest.mark.parametrize("nh,T", [(2, 100), (3, 70), (1, 130), (4, 50)])
 def test_tensor_core_deltaproduct(nh, T):
     cfg = GdnConfig("tcdp", B=1, H=2, T=T, dk=128, dv=128, chunk=64, deltaproduct_nh=nh,
                     s0_std=0.05, seed=2000 + T)
