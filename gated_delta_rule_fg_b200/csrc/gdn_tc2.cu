@@ -651,11 +651,18 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
 #pragma unroll
             for (int j = 0; j < 4; ++j) tc::st16(sm + kA32, off_kmajor(cc, 32 * chh + 8 * j, 1024, 128), tc::f_to_h8(d + 8 * j));
         }
-        {   // Z (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> B operand (K-major, n = r) over T16
+        {   // Z (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> A operand (K-major (m = r, k = r'),
+            // SBO 1024, LBO 128) over T16, and again over P16 (free once Z = P T is done): the
+            // products with Z then run at M = 128 with rows 64-127 repeating rows 0-63, so that their
+            // epilogues use every lane
             if (lane < 16) {
                 const int r = 16 * q + lane;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) tc::st16(sm + kT16, off_kmajor(r, 32 * chh + 8 * j, 1024, 128), tc::f_to_h8(dz + 8 * j));
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 h = tc::f_to_h8(dz + 8 * j);
+                    tc::st16(sm + kT16, off_kmajor(r, 32 * chh + 8 * j, 1024, 128), h);
+                    tc::st16(sm + kP16, off_kmajor(r, 32 * chh + 8 * j, 1024, 128), h);
+                }
             }
         }
     }
@@ -674,7 +681,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
                         idN, kk > 0);
             mma_commit(bar_mma);
         } else if (tid == 32) {       // -Z KG (M = 64; the epilogue adds QG)
-            const uint32_t idQn = idesc_f16(64, 128, false, true, true);
+            const uint32_t idQn = idesc_f16(128, 128, false, true, true);   // [Z; Z]
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), sdesc_sw128(base + kKQ + kk * 2048, 16384, 1024),
@@ -710,11 +717,12 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
             emit(xa, 64 * chh);
             emit(xb, 64 * chh + 32);
         }
-        // Qe = (QG - Z KG) diag(col) (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block
-        // (K-major (m = r, k = c): SBO 2048, LBO 128)
+        // Qe = (QG - Z KG) diag(col) -> block (K-major (m = r, k = c): SBO 2048, LBO 128).  The
+        // product ran at M = 128 with rows repeated, so row r sits in lanes r and 64 + r: warp
+        // (q, chh) takes rows 32 (q % 2) .. +31 and the 32 columns of quarter q / 2 + 2 chh.
         {
             auto emit = [&](float (&x)[32], int c0) {
-                const int r = 16 * q + lane;
+                const int r = 32 * (q & 1) + lane;
 #pragma unroll
                 for (int g8 = 0; g8 < 32; g8 += 8) {
                     float qg[8];
@@ -731,14 +739,10 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
                 for (int g8 = 0; g8 < 32; g8 += 8)
                     *reinterpret_cast<uint4*>(blk + tc::kOffQe + off_kmajor(r, c0 + g8, 2048, 128)) = tc::f_to_h8(x + g8);
             };
-            float xa[32], xb[32];
-            tmem_ld32_async(t0 + lb + 128 + 64 * chh, xa);
-            tmem_ld32_async(t0 + lb + 128 + 64 * chh + 32, xb);
-            tmem_ld_wait2(xa, xb);
-            if (lane < 16) {
-                emit(xa, 64 * chh);
-                emit(xb, 64 * chh + 32);
-            }
+            const int c0 = 32 * ((q >> 1) + 2 * chh);
+            float x[32];
+            tmem_ld32(t0 + lb + 128 + c0, x);
+            emit(x, c0);
         }
     }
     tc_fence_before();
@@ -754,7 +758,7 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
                         idN, kk > 0);
             mma_commit(bar_mma);
         } else if (tid == 32) {       // PU' = Z V
-            const uint32_t idP = idesc_f16(64, 128, false, true);
+            const uint32_t idP = idesc_f16(128, 128, false, true);           // [Z; Z]
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_f16(t0 + 128, sdesc(base + kT16 + kk * 256, 128, 1024), sdesc_sw128(base + kV + kk * 2048, 8192, 1024),
@@ -789,25 +793,21 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
         emit(xa, 64 * chh);
         emit(xb, 64 * chh + 32);
     }
-    if (ok) {   // PU' (M = 64: row r in lane (r % 16) + 32 (r / 16)) -> block (fp16 group-major slices)
+    if (ok) {   // PU' (M = 128, rows repeated; the Qe epilogue's warp split) -> block (fp16 group-major slices)
         const int q = warp & 3, chh = warp >> 2;
         const uint32_t lb = (uint32_t)(32 * q) << 16;
         auto emit = [&](float (&x)[32], int c0) {
-            const int r = 16 * q + lane;
+            const int r = 32 * (q & 1) + lane;
             __half* pu = reinterpret_cast<__half*>(blk + tc::kOffPU) + (size_t)(c0 / NS) * C * NS;
 #pragma unroll
             for (int e = 0; e < 32; ++e) vmax = fmax_nan(vmax, fabsf(x[e]));
 #pragma unroll
             for (int g8 = 0; g8 < 32; g8 += 8) *reinterpret_cast<uint4*>(pu + tc::grp_half(r, g8, C)) = tc::f_to_h8(x + g8);
         };
-        float xa[32], xb[32];
-        tmem_ld32_async(t0 + lb + 128 + 64 * chh, xa);
-        tmem_ld32_async(t0 + lb + 128 + 64 * chh + 32, xb);
-        tmem_ld_wait2(xa, xb);
-        if (lane < 16) {
-            emit(xa, 64 * chh);
-            emit(xb, 64 * chh + 32);
-        }
+        const int c0 = 32 * ((q >> 1) + 2 * chh);
+        float x[32];
+        tmem_ld32(t0 + lb + 128 + c0, x);
+        emit(x, c0);
     }
     if (tid < D) reinterpret_cast<float*>(blk + tc::kOffGC)[tid] = tgam[tid];
     tc_fence_before();
