@@ -91,8 +91,9 @@ __global__ void __launch_bounds__(NT, 2) intra_tma_kernel(Problem p, int cb, int
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);
     // head_fastest: blockIdx.x is the head, so CTAs launched together read the same token rows
-    // (adjacent in memory) for different heads
-    const int c = cb + (head_fastest ? blockIdx.y : blockIdx.x);
+    // (adjacent in memory) for different heads.  Chunks are taken last to first: the blocks the
+    // scan reads first are then the ones written last, still in L2 when it starts.
+    const int c = cb + (head_fastest ? gridDim.y - 1 - blockIdx.y : gridDim.x - 1 - blockIdx.x);
     const int bh = head_fastest ? blockIdx.x : blockIdx.y;
     const int b = bh / p.H, h = bh % p.H;
     const int s0 = c * C;
