@@ -82,9 +82,12 @@ template <typename Tin, int NR, int NI>
 __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
     const int j0 = blockIdx.x * kNS;
     const int bh = blockIdx.y;
-    if (!GDN_IN_BOUNDS(j0 + kNS <= p.dv && bh < p.B * p.H, p.status)) return;
+    // the launcher picks NR = C / 8 and NI = dk / 8, so both are compile-time here (the loops
+    // over rows and channels unroll with constant offsets)
+    constexpr int C = kGroups * NR, dk = kGroups * NI;
+    if (!GDN_IN_BOUNDS(j0 + kNS <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
-    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int dv = p.dv;
     const int tid = threadIdx.x;
     extern __shared__ __align__(16) float sm[];
     float* dS = sm;                          // dk x kNS
@@ -206,14 +209,15 @@ __host__ __device__ inline size_t grad_smem(int C, int dk, int dv) {
                             (size_t)2 * dk * kLd + 2 * C + dk);
 }
 
-// One CTA per (chunk, head).
-template <typename Tin, int RPT>
+// One CTA per (chunk, head).  kC, kDK, kDV: the sizes as compile-time constants (0: read from
+// the problem), so that the common shapes' loops unroll with constant offsets.
+template <typename Tin, int RPT, int kC = 0, int kDK = 0, int kDV = 0>
 __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
-    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;
+    const int C = kC ? kC : p.C, dk = kDK ? kDK : p.dk, dv = kDV ? kDV : p.dv;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H && C == p.C && dk == p.dk && dv == p.dv, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
-    const int C = p.C, dk = p.dk, dv = p.dv;
     const int s0 = c * C;
     const int Cv = min(C, p.L - s0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -566,12 +570,13 @@ cudaError_t launch_rev_nr(const Problem& p, const Grads& gr, cudaStream_t stream
     return cudaErrorInvalidValue;
 }
 
-template <typename Tin, int RPT>
+template <typename Tin, int RPT, int kC = 0, int kDK = 0, int kDV = 0>
 cudaError_t launch_grad(const Problem& p, const Grads& gr, cudaStream_t stream) {
     const size_t s4 = grad_smem(p.C, p.dk, p.dv);
-    const cudaError_t e = cudaFuncSetAttribute(grad_chunk_kernel<Tin, RPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
+    auto kern = grad_chunk_kernel<Tin, RPT, kC, kDK, kDV>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
     if (e != cudaSuccess) return e;
-    grad_chunk_kernel<Tin, RPT><<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
+    kern<<<dim3(p.NC, p.B * p.H), NT, s4, stream>>>(p, gr);
     return cudaGetLastError();
 }
 
@@ -583,6 +588,10 @@ cudaError_t launch_rev_t(const Problem& p, const Grads& gr, cudaStream_t stream)
 
 template <typename Tin>
 cudaError_t launch_grad_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    if (p.dk == 128 && p.dv == 128) {        // d = 128: the sizes as constants
+        if (p.C == 16) return launch_grad<Tin, 8, 16, 128, 128>(p, gr, stream);
+        if (p.C == 32) return launch_grad<Tin, 16, 32, 128, 128>(p, gr, stream);
+    }
     switch (p.C * p.dk / NT) {
         case 2: return launch_grad<Tin, 2>(p, gr, stream);
         case 4: return launch_grad<Tin, 4>(p, gr, stream);

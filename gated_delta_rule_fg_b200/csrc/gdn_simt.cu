@@ -25,15 +25,17 @@ __device__ __forceinline__ float warp_max(float x) {
     return x;
 }
 
-// One CTA per (chunk, head).
-template <typename Tin>
+// One CTA per (chunk, head).  kC, kDK, kDV: the sizes as compile-time constants (0: read from
+// the problem), so that the common shapes' loops unroll with constant offsets.
+template <typename Tin, int kC = 0, int kDK = 0, int kDV = 0>
 __global__ void __launch_bounds__(kSimtThreads)
 intra_simt_kernel(Problem p) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
-    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H, p.status)) return;   // the whole CTA, before any barrier
+    const int C = kC ? kC : p.C, dk = kDK ? kDK : p.dk, dv = kDV ? kDV : p.dv;
+    if (!GDN_IN_BOUNDS(c < p.NC && bh < p.B * p.H && C == p.C && dk == p.dk && dv == p.dv, p.status))
+        return;                                                          // the whole CTA, before any barrier
     const int b = bh / p.H, h = bh % p.H;
-    const int C = p.C, dk = p.dk, dv = p.dv;
     const int s0 = c * C;
     const int Cv = min(C, p.L - s0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -268,9 +270,12 @@ __global__ void __launch_bounds__(kSimtThreads)
 scan_simt_kernel(Problem p) {
     const int j0 = blockIdx.x * kScanCols;
     const int bh = blockIdx.y;
-    if (!GDN_IN_BOUNDS(j0 + kScanCols <= p.dv && bh < p.B * p.H, p.status)) return;
+    // the launcher picks NR = C / kRowGroups and NI = dk / kRowGroups (C and dk are multiples of
+    // it), so both sizes are compile-time here and the loops over them unroll
+    constexpr int C = kRowGroups * NR, dk = kRowGroups * NI;
+    if (!GDN_IN_BOUNDS(j0 + kScanCols <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
-    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int dv = p.dv;
     const int tid = threadIdx.x;
     constexpr int NS = kScanCols;
 
@@ -442,23 +447,28 @@ cudaError_t launch_scan_t(const Problem& p, dim3 grid, size_t smem, cudaStream_t
     return cudaErrorInvalidValue;
 }
 
+template <typename Tin, int kC = 0, int kDK = 0, int kDV = 0>
+cudaError_t launch_intra_k(const Problem& p, size_t smem, cudaStream_t stream) {
+    auto kern = intra_simt_kernel<Tin, kC, kDK, kDV>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<dim3(p.NC, p.B * p.H), kSimtThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_intra_t(const Problem& p, size_t smem, cudaStream_t stream) {
+    if (p.dk == 128 && p.dv == 128) {        // d = 128: the sizes as constants
+        if (p.C == 16) return launch_intra_k<Tin, 16, 128, 128>(p, smem, stream);
+        if (p.C == 32) return launch_intra_k<Tin, 32, 128, 128>(p, smem, stream);
+    }
+    return launch_intra_k<Tin>(p, smem, stream);
+}
+
 cudaError_t launch_simt_intra(const Problem& p, bool bf16, cudaStream_t stream) {
     const size_t s1 = intra_simt_smem(p.C, p.dk, p.dv, p.gdn2_eta != nullptr);
-    if (p.NC > 0) {
-        dim3 g1(p.NC, p.B * p.H);
-        if (bf16) {
-            const cudaError_t e = cudaFuncSetAttribute(intra_simt_kernel<__nv_bfloat16>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
-            if (e != cudaSuccess) return e;
-            intra_simt_kernel<__nv_bfloat16><<<g1, kSimtThreads, s1, stream>>>(p);
-        } else {
-            const cudaError_t e = cudaFuncSetAttribute(intra_simt_kernel<float>,
-                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
-            if (e != cudaSuccess) return e;
-            intra_simt_kernel<float><<<g1, kSimtThreads, s1, stream>>>(p);
-        }
-        return cudaGetLastError();
-    }
+    if (p.NC > 0)
+        return bf16 ? launch_intra_t<__nv_bfloat16>(p, s1, stream) : launch_intra_t<float>(p, s1, stream);
     return cudaSuccess;
 }
 
