@@ -60,8 +60,8 @@ struct Grads {
     float* dS_chunks;            // workspace: dL/dS at every chunk end [B,H,NC,dk,dv]
 };
 
-__host__ __device__ inline size_t rev_smem(int C, int dk) {
-    return sizeof(float) * ((size_t)dk * kNS + (size_t)2 * C * kNS + (size_t)3 * C * dk + dk);
+__host__ __device__ inline size_t rev_smem(int C, int dk, int ns = kNS) {
+    return sizeof(float) * ((size_t)dk * ns + (size_t)2 * C * ns + (size_t)3 * C * dk + dk);
 }
 
 __device__ __forceinline__ void cp16(void* dst, const void* src) {
@@ -74,32 +74,34 @@ __device__ __forceinline__ void cp_floats(float* dst, const float* src, int n, i
 __device__ __forceinline__ void commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void wait_all_but_newest() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// One CTA per (d_v slice, head); serial over chunks from last to first.  Per chunk:
+// One CTA per (d_v slice of NSC columns, head); serial over chunks from last to first.  Per chunk:
 // Y = K' dS' (phase A), then dS = Diag(e^{g_C}) dS' - W^T Y + Qe^T dO (phase B).  The
 // chunk quantities are fetched one phase ahead with asynchronous copies: K' of chunk c-1
 // while phase B of c runs, and W, Qe, e^{g_C}, dO of c-1 while phase A of c-1 runs.
-template <typename Tin, int NR, int NI>
+template <typename Tin, int NR, int NI, int NSC = kNS>
 __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
-    const int j0 = blockIdx.x * kNS;
+    constexpr int kW = NSC;                  // columns of this CTA
+    constexpr int kG = NT / NSC;             // threads per column
+    const int j0 = blockIdx.x * kW;
     const int bh = blockIdx.y;
-    // the launcher picks NR = C / 8 and NI = dk / 8, so both are compile-time here (the loops
+    // the launcher picks NR = C / kG and NI = dk / kG, so both are compile-time here (the loops
     // over rows and channels unroll with constant offsets)
-    constexpr int C = kGroups * NR, dk = kGroups * NI;
-    if (!GDN_IN_BOUNDS(j0 + kNS <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
+    constexpr int C = kG * NR, dk = kG * NI;
+    if (!GDN_IN_BOUNDS(j0 + kW <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
     const int dv = p.dv;
     const int tid = threadIdx.x;
     extern __shared__ __align__(16) float sm[];
-    float* dS = sm;                          // dk x kNS
-    float* Y = dS + (size_t)dk * kNS;        // C x kNS: K' dS'
-    float* dOc = Y + (size_t)C * kNS;        // C x kNS slots: raw dO rows (Tin)
-    float* Wc = dOc + (size_t)C * kNS;       // C x dk
+    float* dS = sm;                          // dk x kW
+    float* Y = dS + (size_t)dk * kW;         // C x kW: K' dS'
+    float* dOc = Y + (size_t)C * kW;         // C x kW slots: raw dO rows (Tin)
+    float* Wc = dOc + (size_t)C * kW;        // C x dk
     float* Qc = Wc + (size_t)C * dk;
     float* Kc = Qc + (size_t)C * dk;
     float* gc = Kc + (size_t)C * dk;         // dk
     const Tin* dO = static_cast<const Tin*>(gr.dO);
     Tin* dOs = reinterpret_cast<Tin*>(dOc);
-    constexpr int kRowChunks = kNS * (int)sizeof(Tin) / 16;   // 16-byte pieces of one row slice
+    constexpr int kRowChunks = kW * (int)sizeof(Tin) / 16;   // 16-byte pieces of one row slice
 
     InterF32 L{C, dk, dv};
     const float* inter = static_cast<const float*>(p.inter);
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
             for (int i = tid; i < C * kRowChunks; i += NT) {
                 const int r = i / kRowChunks, q16 = i % kRowChunks;
                 const int s = c * C + r;
-                Tin* dst = dOs + (size_t)r * kNS;
+                Tin* dst = dOs + (size_t)r * kW;
                 bool ok = false;
                 if (s < p.L) {
                     const RowRef rr = row_ref(p, b, h, s);
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
         commit_group();
     };
 
-    for (int idx = tid; idx < dk * kNS; idx += NT) {
-        const int i = idx / kNS, j = idx % kNS;
+    for (int idx = tid; idx < dk * kW; idx += NT) {
+        const int i = idx / kW, j = idx % kW;
         dS[idx] = gr.dS_final ? gr.dS_final[((size_t)bh * dk + i) * dv + j0 + j] : 0.f;
     }
     fetch_a(p.NC - 1);
@@ -143,26 +145,26 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
         wait_all_but_newest();               // K' of chunk c
         __syncthreads();                     // ... for all; dS' of chunk c is complete
         float* dst = gr.dS_chunks + ((size_t)bh * p.NC + c) * dk * dv;
-        for (int idx = tid; idx < dk * kNS; idx += NT) {
-            const int i = idx / kNS, j = idx % kNS;
+        for (int idx = tid; idx < dk * kW; idx += NT) {
+            const int i = idx / kW, j = idx % kW;
             dst[(size_t)i * dv + j0 + j] = dS[idx];
         }
         {   // thread: column j, rows rg, rg + 8, ...; each dS'[i][j] read once for all its rows
-            const int j = tid % kNS, rg = tid / kNS;
+            const int j = tid % kW, rg = tid / kW;
             float acc[NR];
 #pragma unroll
             for (int m = 0; m < NR; ++m) acc[m] = 0.f;
             for (int i = 0; i < dk; i += 4) {    // K' rows as float4 along i
-                const float x0 = dS[(size_t)i * kNS + j], x1 = dS[(size_t)(i + 1) * kNS + j];
-                const float x2 = dS[(size_t)(i + 2) * kNS + j], x3 = dS[(size_t)(i + 3) * kNS + j];
+                const float x0 = dS[(size_t)i * kW + j], x1 = dS[(size_t)(i + 1) * kW + j];
+                const float x2 = dS[(size_t)(i + 2) * kW + j], x3 = dS[(size_t)(i + 3) * kW + j];
 #pragma unroll
                 for (int m = 0; m < NR; ++m) {
-                    const float4 kk = *reinterpret_cast<const float4*>(Kc + (size_t)(rg + kGroups * m) * dk + i);
+                    const float4 kk = *reinterpret_cast<const float4*>(Kc + (size_t)(rg + kG * m) * dk + i);
                     acc[m] += kk.x * x0 + kk.y * x1 + kk.z * x2 + kk.w * x3;
                 }
             }
 #pragma unroll
-            for (int m = 0; m < NR; ++m) Y[(size_t)(rg + kGroups * m) * kNS + j] = acc[m];
+            for (int m = 0; m < NR; ++m) Y[(size_t)(rg + kG * m) * kW + j] = acc[m];
         }
         __syncthreads();                     // K' buffer free; Y complete
         fetch_a(c - 1);
@@ -171,12 +173,12 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
         // dS <- Diag(gC) dS' - W^T Y + Qe^T dO   (element (i, j) reads only its own dS')
         {   // thread: column j, state rows i0 .. i0 + NI - 1 (contiguous, so the Qe and W rows
             // load as float4); dO[r][j], Y[r][j] read once per r
-            const int j = tid % kNS, i0 = (tid / kNS) * NI;
+            const int j = tid % kW, i0 = (tid / kW) * NI;
             float acc[NI];
 #pragma unroll
-            for (int m = 0; m < NI; ++m) acc[m] = gc[i0 + m] * dS[(size_t)(i0 + m) * kNS + j];
+            for (int m = 0; m < NI; ++m) acc[m] = gc[i0 + m] * dS[(size_t)(i0 + m) * kW + j];
             for (int r = 0; r < C; ++r) {
-                const float d = load_in(dOs, (size_t)r * kNS + j), y = Y[(size_t)r * kNS + j];
+                const float d = load_in(dOs, (size_t)r * kW + j), y = Y[(size_t)r * kW + j];
                 const float4* qv = reinterpret_cast<const float4*>(Qc + (size_t)r * dk + i0);
                 const float4* wv = reinterpret_cast<const float4*>(Wc + (size_t)r * dk + i0);
 #pragma unroll
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
                 }
             }
 #pragma unroll
-            for (int m = 0; m < NI; ++m) dS[(size_t)(i0 + m) * kNS + j] = acc[m];
+            for (int m = 0; m < NI; ++m) dS[(size_t)(i0 + m) * kW + j] = acc[m];
         }
         __syncthreads();                     // W, Qe, e^{g_C}, dO buffers free
         fetch_b(c - 1);
@@ -197,8 +199,8 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (gr.dS0) {
-        for (int idx = tid; idx < dk * kNS; idx += NT) {
-            const int i = idx / kNS, j = idx % kNS;
+        for (int idx = tid; idx < dk * kW; idx += NT) {
+            const int i = idx / kW, j = idx % kW;
             gr.dS0[((size_t)bh * dk + i) * dv + j0 + j] = dS[idx];
         }
     }
@@ -551,12 +553,13 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     }
 }
 
-template <typename Tin, int NR, int NI>
+template <typename Tin, int NR, int NI, int NSC = kNS>
 cudaError_t launch_rev(const Problem& p, const Grads& gr, cudaStream_t stream) {
-    const size_t s3 = rev_smem(p.C, p.dk);
-    const cudaError_t e = cudaFuncSetAttribute(rev_scan_kernel<Tin, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
+    const size_t s3 = rev_smem(p.C, p.dk, NSC);
+    auto kern = rev_scan_kernel<Tin, NR, NI, NSC>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s3);
     if (e != cudaSuccess) return e;
-    rev_scan_kernel<Tin, NR, NI><<<dim3(p.dv / kNS, p.B * p.H), NT, s3, stream>>>(p, gr);
+    kern<<<dim3(p.dv / NSC, p.B * p.H), NT, s3, stream>>>(p, gr);
     return cudaGetLastError();
 }
 
@@ -582,6 +585,12 @@ cudaError_t launch_grad(const Problem& p, const Grads& gr, cudaStream_t stream) 
 
 template <typename Tin>
 cudaError_t launch_rev_t(const Problem& p, const Grads& gr, cudaStream_t stream) {
+    // d_k = 128: slices of 16 columns (16 threads per column), twice the CTAs of 32-column
+    // slices for the same serial chain, each step with half the work
+    if (p.dk == 128) {
+        if (p.C == 16) return launch_rev<Tin, 1, 8, 16>(p, gr, stream);
+        if (p.C == 32) return launch_rev<Tin, 2, 8, 16>(p, gr, stream);
+    }
     return (p.C / kGroups == 2) ? launch_rev_nr<Tin, 2>(p, gr, stream)
          : (p.C / kGroups == 4) ? launch_rev_nr<Tin, 4>(p, gr, stream) : cudaErrorInvalidValue;
 }

@@ -236,8 +236,8 @@ intra_simt_kernel(Problem p) {
 
 // Shared memory of the scan kernel: S (dk x NS), U and the U', PU' slices (C x NS each),
 // W, Qe, K' (C x dk each), e^{g_C} (dk).
-__host__ __device__ inline size_t scan_simt_smem(int C, int dk) {
-    return sizeof(float) * ((size_t)dk * kScanCols + (size_t)3 * C * kScanCols + (size_t)3 * C * dk + dk);
+__host__ __device__ inline size_t scan_simt_smem(int C, int dk, int ns = kScanCols) {
+    return sizeof(float) * ((size_t)dk * ns + (size_t)3 * C * ns + (size_t)3 * C * dk + dk);
 }
 
 // 16-byte asynchronous copy of n floats (n % 4 == 0, both sides 16-byte aligned), spread
@@ -247,37 +247,39 @@ __device__ __forceinline__ void cp_async_floats(float* dst, const float* src, in
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(dst + i)),
                      "l"(src + i) : "memory");
 }
-// Rows of a column slice: rows x 32 floats from a row-major source of row stride ld.
+// Rows of a column slice: rows x NSC floats from a row-major source of row stride ld.
+template <int NSC>
 __device__ __forceinline__ void cp_async_slice(float* dst, const float* src, int rows, int ld, int tid) {
-    for (int i = tid; i < rows * (kScanCols / 4); i += kSimtThreads) {
-        const int r = i / (kScanCols / 4), q4 = i % (kScanCols / 4);
+    for (int i = tid; i < rows * (NSC / 4); i += kSimtThreads) {
+        const int r = i / (NSC / 4), q4 = i % (NSC / 4);
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                     ::"r"((unsigned)__cvta_generic_to_shared(dst + r * kScanCols + 4 * q4)),
+                     ::"r"((unsigned)__cvta_generic_to_shared(dst + r * NSC + 4 * q4)),
                      "l"(src + (size_t)r * ld + 4 * q4) : "memory");
     }
 }
 __device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-// One CTA per (d_v slice of kScanCols columns, head); serial over chunks.  The chunk
+// One CTA per (d_v slice of NSC columns, head); serial over chunks.  The chunk
 // quantities are fetched one phase ahead with asynchronous copies: W, Qe, U', PU' (used
 // only by the U / output phase) for chunk c+1 while the state update of chunk c runs, and
 // K', e^{g_C} (used only by the state update) for chunk c+1 while the U phase of c+1 runs.
 // Every iteration commits both groups (possibly empty), so "all but the newest group have
 // landed" always names the one needed next.
-template <typename Tout, int NR, int NI>
+template <typename Tout, int NR, int NI, int NSC = kScanCols>
 __global__ void __launch_bounds__(kSimtThreads)
 scan_simt_kernel(Problem p) {
-    const int j0 = blockIdx.x * kScanCols;
+    constexpr int NS = NSC;                         // columns of this CTA
+    constexpr int kRG = kSimtThreads / NSC;         // threads per column
+    const int j0 = blockIdx.x * NS;
     const int bh = blockIdx.y;
-    // the launcher picks NR = C / kRowGroups and NI = dk / kRowGroups (C and dk are multiples of
-    // it), so both sizes are compile-time here and the loops over them unroll
-    constexpr int C = kRowGroups * NR, dk = kRowGroups * NI;
-    if (!GDN_IN_BOUNDS(j0 + kScanCols <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
+    // the launcher picks NR = C / kRG and NI = dk / kRG (C and dk are multiples of it), so both
+    // sizes are compile-time here and the loops over them unroll
+    constexpr int C = kRG * NR, dk = kRG * NI;
+    if (!GDN_IN_BOUNDS(j0 + NS <= p.dv && bh < p.B * p.H && p.C == C && p.dk == dk, p.status)) return;
     const int b = bh / p.H, h = bh % p.H;
     const int dv = p.dv;
     const int tid = threadIdx.x;
-    constexpr int NS = kScanCols;
 
     extern __shared__ __align__(16) float sm[];
     float* S = sm;                        // dk x NS
@@ -297,8 +299,8 @@ scan_simt_kernel(Problem p) {
             const float* in = block(c);
             cp_async_floats(Wc, in + L.W(), C * dk, tid);
             cp_async_floats(Qc, in + L.Qe(), C * dk, tid);
-            cp_async_slice(Upc, in + L.Up() + j0, C, dv, tid);
-            cp_async_slice(PUc, in + L.PUp() + j0, C, dv, tid);
+            cp_async_slice<NS>(Upc, in + L.Up() + j0, C, dv, tid);
+            cp_async_slice<NS>(PUc, in + L.PUp() + j0, C, dv, tid);
         }
         cp_async_commit_group();
     };
@@ -339,7 +341,7 @@ scan_simt_kernel(Problem p) {
                     const float sij = S[(size_t)i * NS + j];
 #pragma unroll
                     for (int m = 0; m < NR; ++m) {
-                        const int r = rg + kRowGroups * m;
+                        const int r = rg + kRG * m;
                         ws[m] += Wc[(size_t)r * dk + i] * sij;
                         qs[m] += Qc[(size_t)r * dk + i] * sij;
                     }
@@ -350,7 +352,7 @@ scan_simt_kernel(Problem p) {
                     const float s2 = S[(size_t)(i + 2) * NS + j], s3 = S[(size_t)(i + 3) * NS + j];
 #pragma unroll
                     for (int m = 0; m < NR; ++m) {
-                        const float4 w = *reinterpret_cast<const float4*>(Wc + (size_t)(rg + kRowGroups * m) * dk + i);
+                        const float4 w = *reinterpret_cast<const float4*>(Wc + (size_t)(rg + kRG * m) * dk + i);
                         ws[m] += w.x * s0 + w.y * s1 + w.z * s2 + w.w * s3;
                     }
                 }
@@ -358,7 +360,7 @@ scan_simt_kernel(Problem p) {
 #pragma unroll
             for (int m = 0; m < NR; ++m) {
                 {
-                    const int r = rg + kRowGroups * m;
+                    const int r = rg + kRG * m;
                     const int idx = r * NS + j;
                     U[idx] = Upc[idx] - ws[m];
                     const int s = s0 + r;
@@ -419,11 +421,12 @@ bool simt_supported(int C, int dk, int dv) {
            dv % kScanCols == 0;
 }
 
-template <typename Tout, int NR, int NI>
+template <typename Tout, int NR, int NI, int NSC = kScanCols>
 cudaError_t launch_scan_nr_ni(const Problem& p, dim3 grid, size_t smem, cudaStream_t stream) {
-    const cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<Tout, NR, NI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = scan_simt_kernel<Tout, NR, NI, NSC>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    scan_simt_kernel<Tout, NR, NI><<<grid, kSimtThreads, smem, stream>>>(p);
+    kern<<<grid, kSimtThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -472,7 +475,24 @@ cudaError_t launch_simt_intra(const Problem& p, bool bf16, cudaStream_t stream) 
     return cudaSuccess;
 }
 
+// d_k = 128: slices of 16 columns (16 threads per column), twice the CTAs of 32-column slices
+// for the same serial chain, each step with half the work
+template <typename Tout>
+cudaError_t launch_scan16(const Problem& p, cudaStream_t stream) {
+    constexpr int W = 16, RG = kSimtThreads / W;
+    const size_t smem = scan_simt_smem(p.C, p.dk, W);
+    const dim3 grid(p.dv / W, p.B * p.H);
+    switch (p.C / RG) {
+        case 1: return launch_scan_nr_ni<Tout, 1, 128 / RG, W>(p, grid, smem, stream);
+        case 2: return launch_scan_nr_ni<Tout, 2, 128 / RG, W>(p, grid, smem, stream);
+        case 4: return launch_scan_nr_ni<Tout, 4, 128 / RG, W>(p, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_simt_scan(const Problem& p, bool bf16, cudaStream_t stream) {
+    if (p.dk == 128 && p.dv % 16 == 0)
+        return bf16 ? launch_scan16<__nv_bfloat16>(p, stream) : launch_scan16<float>(p, stream);
     const size_t s2 = scan_simt_smem(p.C, p.dk);
     dim3 g2(p.dv / kScanCols, p.B * p.H);
     return bf16 ? launch_scan_t<__nv_bfloat16>(p, g2, s2, stream) : launch_scan_t<float>(p, g2, s2, stream);
