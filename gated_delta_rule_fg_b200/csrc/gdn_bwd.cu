@@ -72,6 +72,10 @@ __device__ __forceinline__ void cp_floats(float* dst, const float* src, int n, i
     for (int i = 4 * tid; i < n; i += 4 * NT) cp16(dst + i, src + i);
 }
 __device__ __forceinline__ void commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// L2 prefetch of `bytes` (a multiple of 16) from a 16-byte aligned global address
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void wait_all_but_newest() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // One CTA per (d_v slice of NSC columns, head); serial over chunks from last to first.  Per chunk:
@@ -212,9 +216,10 @@ __host__ __device__ inline size_t grad_smem(int C, int dk, int dv) {
 }
 
 // One CTA per (chunk, head).  kC, kDK, kDV: the sizes as compile-time constants (0: read from
-// the problem), so that the common shapes' loops unroll with constant offsets.
+// the problem), so that the common shapes' loops unroll with constant offsets.  At d = 128 the
+// shared memory allows two CTAs per SM, which the register budget is then sized for.
 template <typename Tin, int RPT, int kC = 0, int kDK = 0, int kDV = 0>
-__global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
+__global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Problem p, Grads gr) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
     const int C = kC ? kC : p.C, dk = kDK ? kDK : p.dk, dv = kDV ? kDV : p.dv;
@@ -252,40 +257,70 @@ __global__ void __launch_bounds__(NT) grad_chunk_kernel(Problem p, Grads gr) {
     const float* bvsrc = p.beta_v ? p.beta_v : p.beta;
     const int bvstride = p.beta_v ? dv : dk;
 
-    // 1. rows: q^, k~, v~, log alpha, dO
+    // The chunk's S and dS' (read by phases 3 and 6, each twice) into L2 while the rows and the
+    // Gram products are formed.
+    if (tid == 0) {
+        const size_t n = (size_t)dk * dv;
+        bulk_prefetch_l2(p.S_chunks + ((size_t)bh * p.NC + c) * n, (uint32_t)(n * sizeof(float)));
+        bulk_prefetch_l2(gr.dS_chunks + ((size_t)bh * p.NC + c) * n, (uint32_t)(n * sizeof(float)));
+    }
+    // 1. rows: q^, k~, v~, log alpha, dO.  Every load of a row is issued before any is used (one
+    // round trip to memory per row).
+    constexpr int kJ = 4;                    // channels per lane (d <= 128)
     for (int r = warp; r < C; r += nwarps) {
         float* qr = qh + (size_t)r * dk;
         float* kr = kt + (size_t)r * dk;
         float* gq = g + (size_t)r * dk;
         if (r < Cv) {
             const RowRef rr = row_ref(p, b, h, s0 + r);
-            float ssq = 0.f, ssk = 0.f;
-            for (int j = lane; j < dk; j += 32) {
-                const float xq = load_in(q, rr.tok * dk + j);
-                const float xk = load_in(k, rr.tok * dk + j);
-                qr[j] = xq;
-                kr[j] = xk;
-                ssq += xq * xq;
-                ssk += xk * xk;
+            float xq[kJ], xk[kJ], xa[kJ], xb[kJ], xv[kJ], xo[kJ], xbv[kJ];
+#pragma unroll
+            for (int u = 0; u < kJ; ++u) {
+                const int j = lane + 32 * u;
+                if (j < dk) {
+                    xq[u] = load_in(q, rr.tok * dk + j);
+                    xk[u] = load_in(k, rr.tok * dk + j);
+                    xa[u] = p.alpha_scalar ? 0.f : p.alpha[rr.tok * dk + j];
+                    xb[u] = p.beta_scalar ? 0.f : p.beta[rr.tok * dk + j];
+                }
+                if (j < dv) {
+                    xv[u] = load_in(v, rr.tok * dv + j);
+                    xo[u] = load_in(dO, rr.tok * dv + j);
+                    xbv[u] = p.beta_scalar ? 0.f : bvsrc[rr.tok * bvstride + j];
+                }
             }
+            const float as = p.alpha_scalar ? p.alpha[rr.tok] : 0.f;
+            const float bsr = p.beta_scalar ? p.beta[rr.tok] : 0.f;
+            const float bvr = p.beta_scalar ? bvsrc[rr.tok] : 0.f;
+            float ssq = 0.f, ssk = 0.f;
+#pragma unroll
+            for (int u = 0; u < kJ; ++u)
+                if (lane + 32 * u < dk) {
+                    ssq += xq[u] * xq[u];
+                    ssk += xk[u] * xk[u];
+                }
             const float a = rsqrtf(warp_sum(ssq) + kNormEps);
             const float bk = rsqrtf(warp_sum(ssk) + kNormEps);
             if (lane == 0) {
                 iq[r] = a;
                 ik[r] = bk;
             }
-            const float bs = p.beta_scalar ? sqrtf(p.beta[rr.tok]) : 0.f;
-            const float la = p.alpha_scalar ? logf(p.alpha[rr.tok]) : 0.f;
-            for (int j = lane; j < dk; j += 32) {
-                qr[j] *= a;
-                kr[j] *= bk * (p.beta_scalar ? bs : sqrtf(p.beta[rr.tok * dk + j]));
-                gq[j] = p.alpha_scalar ? la : logf(p.alpha[rr.tok * dk + j]);
-            }
-            const float bvs = p.beta_scalar ? sqrtf(bvsrc[rr.tok]) : 0.f;
-            for (int j = lane; j < dv; j += 32) {
-                const float sb = p.beta_scalar ? bvs : sqrtf(bvsrc[rr.tok * bvstride + j]);
-                vt[(size_t)r * dv + j] = load_in(v, rr.tok * dv + j) * sb;
-                dOs[(size_t)r * dv + j] = load_in(dO, rr.tok * dv + j);
+            const float bs = p.beta_scalar ? sqrtf(bsr) : 0.f;
+            const float la = p.alpha_scalar ? logf(as) : 0.f;
+            const float bvs = p.beta_scalar ? sqrtf(bvr) : 0.f;
+#pragma unroll
+            for (int u = 0; u < kJ; ++u) {
+                const int j = lane + 32 * u;
+                if (j < dk) {
+                    qr[j] = xq[u] * a;
+                    kr[j] = xk[u] * (bk * (p.beta_scalar ? bs : sqrtf(xb[u])));
+                    gq[j] = p.alpha_scalar ? la : logf(xa[u]);
+                }
+                if (j < dv) {
+                    const float sb = p.beta_scalar ? bvs : sqrtf(xbv[u]);
+                    vt[(size_t)r * dv + j] = xv[u] * sb;
+                    dOs[(size_t)r * dv + j] = xo[u];
+                }
             }
         } else {
             for (int j = lane; j < dk; j += 32) { qr[j] = 0.f; kr[j] = 0.f; gq[j] = 0.f; }
