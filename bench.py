@@ -414,8 +414,7 @@ def main():
     ap.add_argument("--H", type=int, default=None, help="override the workload's heads")
     ap.add_argument("--T", type=int, default=None, help="override the workload's tokens per sequence")
     ap.add_argument("--chunk", type=int, default=None,
-                    help="override the chunk length (the backward's default, 16, is its faster supported "
-                         "one: 27.1 ms against 40.3 ms for chunk 32 at the 32K prefill)")
+                    help="override the chunk length (the backward's default is 16)")
     args = ap.parse_args()
     cfg = CONFIGS[args.workload]
     over = {k: getattr(args, k) for k in ("B", "H", "T") if getattr(args, k) is not None}
