@@ -373,19 +373,37 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
             dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
         }
         __syncthreads();
-        for (int idx = tid; idx < C * kNS; idx += NT) {
-            const int r = idx / kNS, jj = idx % kNS;
-            float ks = 0.f, kd = 0.f;
-            for (int i = 0; i < dk; i += 4) {    // K_G, K_E rows as float4 along i
-                const float4 g4 = *reinterpret_cast<const float4*>(KG + (size_t)r * dk + i);
-                const float4 e4 = *reinterpret_cast<const float4*>(KE + (size_t)r * dk + i);
-                ks += g4.x * St[i * kLd + jj] + g4.y * St[(i + 1) * kLd + jj] +
-                      g4.z * St[(i + 2) * kLd + jj] + g4.w * St[(i + 3) * kLd + jj];
-                kd += e4.x * dSt[i * kLd + jj] + e4.y * dSt[(i + 1) * kLd + jj] +
-                      e4.z * dSt[(i + 2) * kLd + jj] + e4.w * dSt[(i + 3) * kLd + jj];
+        {   // thread: column jj, rows r0, r0 + 8, ... (C / 8 of them, at most 4); each S and dS'
+            // element is read once for all of them, K_G and K_E rows as float4 along i
+            constexpr int kMaxRows = 4, kRowStep = NT / kNS;
+            const int jj = tid % kNS, r0 = tid / kNS, nr = C / kRowStep;
+            float ks[kMaxRows], kd[kMaxRows];
+#pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) { ks[m] = 0.f; kd[m] = 0.f; }
+            for (int i = 0; i < dk; i += 4) {
+                const float s0 = St[i * kLd + jj], s1 = St[(i + 1) * kLd + jj];
+                const float s2 = St[(i + 2) * kLd + jj], s3 = St[(i + 3) * kLd + jj];
+                const float d0 = dSt[i * kLd + jj], d1 = dSt[(i + 1) * kLd + jj];
+                const float d2 = dSt[(i + 2) * kLd + jj], d3 = dSt[(i + 3) * kLd + jj];
+#pragma unroll
+                for (int m = 0; m < kMaxRows; ++m) {
+                    if (m < nr) {
+                        const size_t ro = (size_t)(r0 + kRowStep * m) * dk + i;
+                        const float4 g4 = *reinterpret_cast<const float4*>(KG + ro);
+                        const float4 e4 = *reinterpret_cast<const float4*>(KE + ro);
+                        ks[m] = fmaf(g4.w, s3, fmaf(g4.z, s2, fmaf(g4.y, s1, fmaf(g4.x, s0, ks[m]))));
+                        kd[m] = fmaf(e4.w, d3, fmaf(e4.z, d2, fmaf(e4.y, d1, fmaf(e4.x, d0, kd[m]))));
+                    }
+                }
             }
-            U[(size_t)r * dv + jt + jj] = vt[(size_t)r * dv + jt + jj] - ks;
-            dR[(size_t)r * dv + jt + jj] = kd;
+#pragma unroll
+            for (int m = 0; m < kMaxRows; ++m) {
+                if (m < nr) {
+                    const size_t o = (size_t)(r0 + kRowStep * m) * dv + jt + jj;
+                    U[o] = vt[o] - ks[m];
+                    dR[o] = kd[m];
+                }
+            }
         }
         __syncthreads();
     }
@@ -484,9 +502,9 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
                 const float4 a = *reinterpret_cast<const float4*>(dOs + o);
                 const float4 rr4 = *reinterpret_cast<const float4*>(dR + o);
                 const float4 u = *reinterpret_cast<const float4*>(U + o);
-                G1[m] += a.x * sv[0] + a.y * sv[1] + a.z * sv[2] + a.w * sv[3];
-                G2[m] += rr4.x * sv[0] + rr4.y * sv[1] + rr4.z * sv[2] + rr4.w * sv[3];
-                G3[m] += u.x * dv4[0] + u.y * dv4[1] + u.z * dv4[2] + u.w * dv4[3];
+                G1[m] = fmaf(a.w, sv[3], fmaf(a.z, sv[2], fmaf(a.y, sv[1], fmaf(a.x, sv[0], G1[m]))));
+                G2[m] = fmaf(rr4.w, sv[3], fmaf(rr4.z, sv[2], fmaf(rr4.y, sv[1], fmaf(rr4.x, sv[0], G2[m]))));
+                G3[m] = fmaf(u.w, dv4[3], fmaf(u.z, dv4[2], fmaf(u.y, dv4[1], fmaf(u.x, dv4[0], G3[m]))));
             }
         }
     }
