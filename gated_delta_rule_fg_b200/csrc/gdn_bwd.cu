@@ -444,16 +444,10 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
         }
         __syncthreads();
     }
-    // 4. U = (I + A)^{-1} R (forward substitution); dU = K_E dS' + P^T dO;
-    //    dR = (I + A)^{-T} dU (back substitution)
-    for (int r = 1; r < C; ++r) {
-        for (int j = tid; j < dv; j += NT) {
-            float acc = U[(size_t)r * dv + j];
-            for (int i = 0; i < r; ++i) acc -= A[(size_t)r * C + i] * U[(size_t)i * dv + j];
-            U[(size_t)r * dv + j] = acc;
-        }
-        __syncthreads();
-    }
+    // 4. dU = K_E dS' + P^T dO, then U = (I + A)^{-1} R (forward substitution) and
+    //    dR = (I + A)^{-T} dU (back substitution).  Each substitution runs down one column per
+    //    thread, in registers: threads 0 .. NT/2 - 1 take U's columns, the others dR's (the two
+    //    are independent), so no barrier is needed between rows.
     for (int idx = tid; idx < C * dv; idx += NT) {
         const int i = idx / dv, j = idx % dv;
         float acc = dR[idx];
@@ -461,14 +455,44 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
         dR[idx] = acc;
     }
     __syncthreads();
-    for (int r = C - 2; r >= 0; --r) {
-        for (int j = tid; j < dv; j += NT) {
-            float acc = dR[(size_t)r * dv + j];
-            for (int i = r + 1; i < C; ++i) acc -= A[(size_t)i * C + r] * dR[(size_t)i * dv + j];
-            dR[(size_t)r * dv + j] = acc;
+    {
+        constexpr int kMaxC = kC ? kC : 32;  // rows (the chunk; at most 32)
+        constexpr int half = NT / 2;
+        const bool second = tid >= half;
+        float* X = second ? dR : U;
+        for (int j = second ? tid - half : tid; j < dv; j += half) {
+            float x[kMaxC];
+#pragma unroll
+            for (int r = 0; r < kMaxC; ++r)
+                if (r < C) x[r] = X[(size_t)r * dv + j];
+            if (!second) {
+#pragma unroll
+                for (int r = 1; r < kMaxC; ++r) {
+                    if (r < C) {
+                        float acc = x[r];
+#pragma unroll
+                        for (int i = 0; i < r; ++i) acc -= A[(size_t)r * C + i] * x[i];
+                        x[r] = acc;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int r = kMaxC - 2; r >= 0; --r) {
+                    if (r <= C - 2) {
+                        float acc = x[r];
+#pragma unroll
+                        for (int i = r + 1; i < kMaxC; ++i)
+                            if (i < C) acc -= A[(size_t)i * C + r] * x[i];
+                        x[r] = acc;
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kMaxC; ++r)
+                if (r < C) X[(size_t)r * dv + j] = x[r];
         }
-        __syncthreads();
     }
+    __syncthreads();
     // 5. dP = lower(dO U^T), dA = strictly-lower(-dR U^T).  Where U^T (rows padded to C + 1)
     //    fits the free tile buffers: one thread per (r, i) pair with no cross-lane reduction
     //    (a warp's lanes read consecutive i of U^T; dO and dR rows are broadcasts); otherwise
