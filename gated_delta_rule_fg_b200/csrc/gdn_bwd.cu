@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
 #pragma unroll
                 for (int m = 0; m < NR; ++m) {
                     const float4 kk = *reinterpret_cast<const float4*>(Kc + (size_t)(rg + kG * m) * dk + i);
-                    acc[m] += kk.x * x0 + kk.y * x1 + kk.z * x2 + kk.w * x3;
+                    acc[m] = fmaf(kk.w, x3, fmaf(kk.z, x2, fmaf(kk.y, x1, fmaf(kk.x, x0, acc[m]))));
                 }
             }
 #pragma unroll
@@ -188,10 +188,10 @@ __global__ void __launch_bounds__(NT) rev_scan_kernel(Problem p, Grads gr) {
 #pragma unroll
                 for (int m4 = 0; m4 < NI / 4; ++m4) {
                     const float4 qq = qv[m4], ww = wv[m4];
-                    acc[4 * m4 + 0] += qq.x * d - ww.x * y;
-                    acc[4 * m4 + 1] += qq.y * d - ww.y * y;
-                    acc[4 * m4 + 2] += qq.z * d - ww.z * y;
-                    acc[4 * m4 + 3] += qq.w * d - ww.w * y;
+                    acc[4 * m4 + 0] = fmaf(-ww.x, y, fmaf(qq.x, d, acc[4 * m4 + 0]));
+                    acc[4 * m4 + 1] = fmaf(-ww.y, y, fmaf(qq.y, d, acc[4 * m4 + 1]));
+                    acc[4 * m4 + 2] = fmaf(-ww.z, y, fmaf(qq.z, d, acc[4 * m4 + 2]));
+                    acc[4 * m4 + 3] = fmaf(-ww.w, y, fmaf(qq.w, d, acc[4 * m4 + 3]));
                 }
             }
 #pragma unroll

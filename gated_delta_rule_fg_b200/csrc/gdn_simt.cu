@@ -353,7 +353,7 @@ scan_simt_kernel(Problem p) {
 #pragma unroll
                     for (int m = 0; m < NR; ++m) {
                         const float4 w = *reinterpret_cast<const float4*>(Wc + (size_t)(rg + kRG * m) * dk + i);
-                        ws[m] += w.x * s0 + w.y * s1 + w.z * s2 + w.w * s3;
+                        ws[m] = fmaf(w.w, s3, fmaf(w.z, s2, fmaf(w.y, s1, fmaf(w.x, s0, ws[m]))));
                     }
                 }
             }
