@@ -151,39 +151,90 @@ intra_simt_kernel(Problem p) {
     }
     __syncthreads();
 
-    // 3. A (i < r) and P (i <= r) with the decay formed element by element.
-    for (int pr = warp; pr < C * C; pr += nwarps) {
-        const int r = pr / C, i = pr % C;
-        float a = 0.f, pp = 0.f;
-        if (i <= r) {
-            for (int j = lane; j < dk; j += 32) {
-                const float e = expf(g[(size_t)r * dk + j] - g[(size_t)i * dk + j]);
-                const float ke = kt[(size_t)i * dk + j] * e;
-                pp += qh[(size_t)r * dk + j] * ke;
-                a += ew[(size_t)r * dk + j] * ke;
+    // 3. A (i < r) and P (i <= r) with the decay formed element by element.  Warp w takes rows
+    // 16 m + w and 16 m + 15 - w (the same number of pairs for every warp); its lanes run over
+    // channels and hold the partial sums of 16 A and 16 P entries at a time, which one butterfly
+    // of 31 shuffles reduces (lane l ends with entry l; the same pairing as a warp sum per entry).
+    {
+        const unsigned full = 0xffffffffu;
+        constexpr int kJ = 4;                // channels per lane (d <= 128)
+        for (int k = 0; k < C / 8; ++k) {
+            const int r = 16 * (k >> 1) + ((k & 1) ? 15 - warp : warp);
+            float er_[kJ], qr_[kJ], gr_[kJ];
+#pragma unroll
+            for (int u = 0; u < kJ; ++u) {
+                const int j = lane + 32 * u;
+                if (j < dk) {
+                    er_[u] = ew[(size_t)r * dk + j];
+                    qr_[u] = qh[(size_t)r * dk + j];
+                    gr_[u] = g[(size_t)r * dk + j];
+                }
             }
-            a = warp_sum(a);
-            pp = warp_sum(pp);
-        }
-        if (lane == 0) {
-            A[pr] = (i < r) ? a : 0.f;
-            P[pr] = pp;
+            for (int ih = 0; ih < C; ih += 16) {
+                float v[32];                 // v[t]: A[r][ih + t], v[16 + t]: P[r][ih + t]
+#pragma unroll
+                for (int t = 0; t < 32; ++t) v[t] = 0.f;
+                if (ih <= r) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const int i = ih + t;
+                        if (i <= r) {
+#pragma unroll
+                            for (int u = 0; u < kJ; ++u) {
+                                const int j = lane + 32 * u;
+                                if (j < dk) {
+                                    const float e = expf(gr_[u] - g[(size_t)i * dk + j]);
+                                    const float ke = kt[(size_t)i * dk + j] * e;
+                                    v[16 + t] += qr_[u] * ke;
+                                    v[t] += er_[u] * ke;
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1) {
+                        const bool upper = (lane & off) != 0;
+#pragma unroll
+                        for (int t = 0; t < off; ++t) {
+                            const float send = upper ? v[t] : v[t + off];
+                            const float keep = upper ? v[t + off] : v[t];
+                            v[t] = keep + __shfl_xor_sync(full, send, off);
+                        }
+                    }
+                }
+                const int i = ih + (lane & 15);
+                if (lane < 16) A[(size_t)r * C + i] = (i < r) ? v[0] : 0.f;
+                else P[(size_t)r * C + i] = (i <= r) ? v[0] : 0.f;
+            }
         }
     }
     __syncthreads();
 
-    // 4. T = (I + A)^{-1} by forward substitution, one row at a time:
+    // 4. T = (I + A)^{-1} by forward substitution, one column per thread in registers:
     //    T[r][j] = delta_rj - sum_{j <= i < r} A[r][i] T[i][j].
-    for (int r = 0; r < C; ++r) {
-        for (int j = tid; j < C; j += kSimtThreads) {
-            float acc = (j == r) ? 1.f : 0.f;
-            if (j < r) {
-                for (int i = j; i < r; ++i) acc -= A[(size_t)r * C + i] * Tm[(size_t)i * C + j];
+    {
+        constexpr int kMaxC = kC ? kC : 64;  // rows (the chunk; at most 64)
+        const int j = tid;
+        if (j < C) {
+            float t[kMaxC];
+#pragma unroll
+            for (int r = 0; r < kMaxC; ++r) {
+                if (r < C) {
+                    float acc = (j == r) ? 1.f : 0.f;
+                    if (j < r) {
+#pragma unroll
+                        for (int i = 0; i < r; ++i)
+                            if (i >= j) acc -= A[(size_t)r * C + i] * t[i];
+                    }
+                    t[r] = acc;
+                }
             }
-            Tm[(size_t)r * C + j] = acc;
+#pragma unroll
+            for (int r = 0; r < kMaxC; ++r)
+                if (r < C) Tm[(size_t)r * C + j] = t[r];
         }
-        __syncthreads();
     }
+    __syncthreads();
 
     // 5. chunk-end decay, K', and the e^g-scaled operands.
     InterF32 L{C, dk, dv};
