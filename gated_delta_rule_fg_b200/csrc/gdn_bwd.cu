@@ -402,14 +402,38 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
 
     const float* Sg = p.S_chunks + ((size_t)bh * p.NC + c) * dk * dv;
     const float* dSg = gr.dS_chunks + ((size_t)bh * p.NC + c) * dk * dv;
-    // 3. R = V~ - K_G S and K_E dS', tile by tile over d_v
-    for (int jt = 0; jt < dv; jt += kNS) {
-        for (int idx = tid; idx < dk * kNS; idx += NT) {
-            const int i = idx / kNS, jj = idx % kNS;
-            St[i * kLd + jj] = Sg[(size_t)i * dv + jt + jj];
-            dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
+    // A dk x kNS tile of S and dS' (columns jt ..): this thread's share, loaded into registers
+    // one tile ahead of its use (the load is in flight while the previous tile is worked on)
+    constexpr int kTV = (kDK ? kDK : 128) * kNS / NT;     // values per thread (dk <= 128)
+    float ts[kTV], tds[kTV];
+    auto tile_load = [&](int jt) {
+#pragma unroll
+        for (int m = 0; m < kTV; ++m) {
+            const int idx = tid + m * NT;
+            if (idx < dk * kNS) {
+                const int i = idx / kNS, jj = idx % kNS;
+                ts[m] = Sg[(size_t)i * dv + jt + jj];
+                tds[m] = dSg[(size_t)i * dv + jt + jj];
+            }
         }
+    };
+    auto tile_store = [&]() {
+#pragma unroll
+        for (int m = 0; m < kTV; ++m) {
+            const int idx = tid + m * NT;
+            if (idx < dk * kNS) {
+                const int i = idx / kNS, jj = idx % kNS;
+                St[i * kLd + jj] = ts[m];
+                dSt[i * kLd + jj] = tds[m];
+            }
+        }
+    };
+    // 3. R = V~ - K_G S and K_E dS', tile by tile over d_v
+    tile_load(0);
+    for (int jt = 0; jt < dv; jt += kNS) {
+        tile_store();
         __syncthreads();
+        if (jt + kNS < dv) tile_load(jt + kNS);
         {   // thread: column jj, rows r0, r0 + 8, ... (C / 8 of them, at most 4); each S and dS'
             // element is read once for all of them, K_G and K_E rows as float4 along i
             constexpr int kMaxRows = 4, kRowStep = NT / kNS;
@@ -541,14 +565,12 @@ __global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Prob
     float G1[RPT], G2[RPT], G3[RPT], G4 = 0.f;
 #pragma unroll
     for (int m = 0; m < RPT; ++m) { G1[m] = 0.f; G2[m] = 0.f; G3[m] = 0.f; }
+    tile_load(0);
     for (int jt = 0; jt < dv; jt += kNS) {
         __syncthreads();
-        for (int idx = tid; idx < dk * kNS; idx += NT) {
-            const int i = idx / kNS, jj = idx % kNS;
-            St[i * kLd + jj] = Sg[(size_t)i * dv + jt + jj];
-            dSt[i * kLd + jj] = dSg[(size_t)i * dv + jt + jj];
-        }
+        tile_store();
         __syncthreads();
+        if (jt + kNS < dv) tile_load(jt + kNS);
         for (int jj = 0; jj < kNS; jj += 4) {   // four columns at a time: row data as float4
             float sv[4], dv4[4];
 #pragma unroll
