@@ -216,10 +216,11 @@ __host__ __device__ inline size_t grad_smem(int C, int dk, int dv) {
 }
 
 // One CTA per (chunk, head).  kC, kDK, kDV: the sizes as compile-time constants (0: read from
-// the problem), so that the common shapes' loops unroll with constant offsets.  At d = 128 the
-// shared memory allows two CTAs per SM, which the register budget is then sized for.
+// the problem), so that the common shapes' loops unroll with constant offsets.  At d = 128 and
+// chunk 16 the shared memory allows two CTAs per SM, which the register budget is then sized
+// for (at chunk 32 it allows one).
 template <typename Tin, int RPT, int kC = 0, int kDK = 0, int kDV = 0>
-__global__ void __launch_bounds__(NT, kDK == 128 ? 2 : 1) grad_chunk_kernel(Problem p, Grads gr) {
+__global__ void __launch_bounds__(NT, (kDK == 128 && kC == 16) ? 2 : 1) grad_chunk_kernel(Problem p, Grads gr) {
     const int c = blockIdx.x;
     const int bh = blockIdx.y;
     const int C = kC ? kC : p.C, dk = kDK ? kDK : p.dk, dv = kDV ? kDV : p.dv;
